@@ -1,0 +1,245 @@
+/*
+ * zimage_dit.h -- C ABI of the B200 (sm_100a) Z-Image S3-DiT forward library.
+ *
+ * What it computes (page title, section):
+ *   - ostris ai-toolkit docs "Z-Image", sections "Architecture" and "Latent
+ *     space": a single-stream DiT; text and 2x2-patchified image tokens share
+ *     one sequence; 2 noise-refiner blocks (image tokens), 2 context-refiner
+ *     blocks (text tokens, unmodulated) and 30 main blocks; hidden 3840 =
+ *     30 heads x 128; SwiGLU FFN 10240; RMSNorm and QK-RMSNorm; 3-axis RoPE
+ *     [32, 48, 48] with theta 256; adaLN modulation from a 256-d timestep
+ *     embedding.
+ *   - z-image-turbo-mnn model card, "Conversion details": the attention output
+ *     projection and FFN w2 feed an RMSNorm directly (post-norms); "Model
+ *     files": transformer(sample [1,16,H/8,W/8], timestep [1], text features
+ *     [1,L,2560]) -> output of the sample's shape; "Scheduler": FlowMatch
+ *     Euler with shift 3.0, sigmas linspace(1, 1/N, N) shifted, timestep
+ *     passed as 1 - sigma, model output negated before the Euler step.
+ *   - FastVideo zimage handoff, "Pinned official pipeline context": a
+ *     num_steps + 1 schedule ending at sigma 0, the final zero-sigma call skipped.
+ * Readings of points the pages leave open are fixed in the library and listed
+ * in the design notes; the same readings define the CPU oracle in the tests.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless the argument name starts
+ *     with h_.  The caller owns every buffer and the stream; the library never
+ *     allocates or frees device memory and never synchronises the stream.
+ *     Pointers must stay valid until the enqueued work has completed.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  Weights are row-major
+ *     in the checkpoint's [out, in] orientation.
+ *   - Device pointers to bf16 matrices and to fp32 activations must be 16-byte
+ *     aligned (TMA and vector loads); otherwise ZI_ERR_ALIGN.
+ *   - Every call validates its arguments before enqueuing anything and returns
+ *     a status (0 = ZI_OK, negative = error); nothing is enqueued on error.
+ *     Asynchronous device failures (a pipeline wait that ran out) are reported
+ *     later by zi_device_status().
+ *   - There is no CPU fallback: calls that launch kernels fail with
+ *     ZI_ERR_DEVICE unless the current device is compute capability 10.0.
+ */
+#ifndef ZIMAGE_DIT_H
+#define ZIMAGE_DIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZI_API __attribute__((visibility("default")))
+#else
+#define ZI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st* zi_stream_t;
+
+enum zi_status {
+  ZI_OK = 0,
+  ZI_ERR_ARG = -1,       /* null pointer, bad enum, negative size */
+  ZI_ERR_SHAPE = -2,     /* sizes the kernels do not support */
+  ZI_ERR_ALIGN = -3,     /* pointer or stride not 16-byte aligned */
+  ZI_ERR_WORKSPACE = -4, /* workspace missing or smaller than zi_*_workspace_size() */
+  ZI_ERR_CUDA = -5,      /* a CUDA runtime/driver call failed (launch error etc.) */
+  ZI_ERR_TIMEOUT = -6,   /* a kernel's bounded pipeline wait ran out (zi_device_status) */
+  ZI_ERR_DEVICE = -7     /* current device is not an sm_100 GPU */
+};
+
+/* Sizes of one model variant.  zi_config_default() gives Z-Image's
+ * (ostris "Z-Image", "Architecture"; numbers checked against the 6.15B /
+ * 521-key totals of "Components" and the FastVideo "Transformer" notes). */
+typedef struct zi_config {
+  int dim;          /* D, hidden width (3840); multiple of 256 */
+  int heads;        /* attention heads (30); dim == heads * head_dim */
+  int head_dim;     /* 128 (the only supported value) */
+  int ffn;          /* SwiGLU inner width F (10240) */
+  int cap_dim;      /* text-feature width (2560) */
+  int t_freq;       /* sinusoidal timestep width (256) */
+  int t_mid;        /* timestep MLP hidden width (1024) */
+  int in_ch;        /* latent channels (16) */
+  int patch;        /* 2 (the only supported value) */
+  int n_noise;      /* noise-refiner blocks (2) */
+  int n_ctx;        /* context-refiner blocks (2) */
+  int n_main;       /* main blocks (30) */
+  int rope_axes[3]; /* {32, 48, 48}; sum == head_dim, each even */
+  float rope_theta; /* 256 */
+  float norm_eps;   /* every RMSNorm (1e-5) */
+  float final_eps;  /* final LayerNorm (1e-6) */
+  float t_scale;    /* model timestep t in [0,1] is scaled by this (1000) before the sinusoid */
+} zi_config;
+
+/* Weights of one block (device pointers, bf16).  D = dim, F = ffn,
+ * Fp = ffn rounded up to a multiple of 128 (zi_ffn_padded). */
+typedef struct zi_block_weights {
+  const uint16_t* w_qkv;   /* [3D, D]: rows of to_q, then to_k, then to_v (zi_pack_qkv) */
+  const uint16_t* w_out;   /* [D, D]  attention output projection */
+  const uint16_t* w13;     /* [2Fp, D]: w1 and w3 interleaved in 128-row groups (zi_pack_ffn) */
+  const uint16_t* w2;      /* [D, Fp]: w2 with zero columns F..Fp (zi_pack_ffn) */
+  const uint16_t* g_attn1; /* [D] pre-attention RMSNorm gain */
+  const uint16_t* g_attn2; /* [D] post-attention RMSNorm gain */
+  const uint16_t* g_ffn1;  /* [D] pre-FFN RMSNorm gain */
+  const uint16_t* g_ffn2;  /* [D] post-FFN RMSNorm gain */
+  const uint16_t* g_q;     /* [head_dim] QK-RMSNorm gains, shared by all heads */
+  const uint16_t* g_k;     /* [head_dim] */
+  const uint16_t* w_ada;   /* [4D, min(D,256)] adaLN linear, or NULL for an unmodulated block */
+  const uint16_t* b_ada;   /* [4D] its bias (NULL iff w_ada is NULL) */
+} zi_block_weights;
+
+/* Weights of the whole transformer.  The block arrays are HOST arrays (of
+ * structs holding device pointers) of n_noise / n_ctx / n_main entries. */
+typedef struct zi_model_weights {
+  const uint16_t* x_emb_w;   /* [D, 4*in_ch]  x_embedder */
+  const uint16_t* x_emb_b;   /* [D] */
+  const uint16_t* cap_norm;  /* [cap_dim]  cap_embedder RMSNorm gain */
+  const uint16_t* cap_w;     /* [D, cap_dim] */
+  const uint16_t* cap_b;     /* [D] */
+  const uint16_t* t_w1;      /* [t_mid, t_freq] */
+  const uint16_t* t_b1;      /* [t_mid] */
+  const uint16_t* t_w2;      /* [min(D,256), t_mid] */
+  const uint16_t* t_b2;      /* [min(D,256)] */
+  const uint16_t* final_ada_w; /* [D, min(D,256)] final layer adaLN (applied to SiLU(c)) */
+  const uint16_t* final_ada_b; /* [D] */
+  const uint16_t* final_w;   /* [4*in_ch, D] final_layer.linear */
+  const uint16_t* final_b;   /* [4*in_ch] */
+  const zi_block_weights* noise; /* host array [n_noise], modulated */
+  const zi_block_weights* ctx;   /* host array [n_ctx], w_ada == NULL */
+  const zi_block_weights* main;  /* host array [n_main], modulated */
+} zi_model_weights;
+
+/* Human-readable text of a status code (static storage). */
+ZI_API const char* zi_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+ZI_API int zi_version(void);
+
+/* Fill *cfg with Z-Image's sizes (see zi_config).  ZI_ERR_ARG if cfg is NULL. */
+ZI_API int zi_config_default(zi_config* cfg);
+
+/* ffn rounded up to a multiple of 128 (the interleave group of w13). */
+ZI_API int zi_ffn_padded(int ffn);
+
+/* ---------------------------------------------------------------- weight layout
+ * Library-owned layout steps, enqueued on `stream` as device copies. */
+
+/* w_qkv[0:D] = wq, [D:2D] = wk, [2D:3D] = wv; each [D, D]. */
+ZI_API int zi_pack_qkv(const uint16_t* wq, const uint16_t* wk, const uint16_t* wv, int dim, uint16_t* w_qkv,
+                zi_stream_t stream);
+
+/* w13 [2Fp, D]: group g (128 rows) of w1 goes to rows [256g, 256g+128) and
+ * group g of w3 to rows [256g+128, 256g+256); rows past F in a group are zero.
+ * w2p [D, Fp] = w2 [D, F] with zero columns F..Fp.  Lets one 256-wide GEMM
+ * tile hold matching gate and up columns for the fused SwiGLU. */
+ZI_API int zi_pack_ffn(const uint16_t* w1, const uint16_t* w3, const uint16_t* w2, int ffn, int dim, uint16_t* w13,
+                uint16_t* w2p, zi_stream_t stream);
+
+/* ---------------------------------------------------------------- workspaces */
+
+/* Bytes of workspace zi_block_forward needs for batch x seq tokens. */
+ZI_API int zi_block_workspace_size(const zi_config* cfg, int batch, int seq, size_t* h_bytes);
+
+/* Bytes of workspace zi_model_forward needs for batch x (s_img + s_txt) tokens,
+ * s_img = (lat_h/2)(lat_w/2). */
+ZI_API int zi_model_workspace_size(const zi_config* cfg, int batch, int lat_h, int lat_w, int s_txt, size_t* h_bytes);
+
+/* ---------------------------------------------------------------- the forward */
+
+/* One S3-DiT block (ostris "Z-Image", "Architecture"; post-norms per the
+ * z-image-turbo-mnn card, "Conversion details") on x [batch, seq, D] fp32:
+ *   h = RMSNorm1(x)(1 + scale_msa); q, k, v = h Wqkv; q, k <- RoPE(QKRMSNorm(.));
+ *   x += tanh(gate_msa) RMSNorm2(Attn(q, k, v) Wout);
+ *   h = RMSNormF1(x)(1 + scale_mlp); x += tanh(gate_mlp) RMSNormF2(W2(SiLU(W1 h) * W3 h)),
+ * with [scale_msa, gate_msa, scale_mlp, gate_mlp] = w_ada c + b_ada.
+ * Unmodulated blocks (w->w_ada == NULL) use scale 0 and gate 1; d_c may then be NULL.
+ *   d_c    fp32 [batch, min(D,256)] conditioning vector (t-embedder output)
+ *   d_pos  int32 [seq, 3] position ids of one sequence (shared by the batch)
+ *   d_x_in / d_x_out  fp32 [batch, seq, D]; may be the same buffer
+ *   d_ws   workspace of at least zi_block_workspace_size() bytes (256-byte aligned)
+ * Attention is non-causal over the seq tokens of each batch element. */
+ZI_API int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const float* d_c, const int32_t* d_pos,
+                     int batch, int seq, const float* d_x_in, float* d_x_out, void* d_ws, size_t ws_bytes,
+                     zi_stream_t stream);
+
+/* Full transformer forward (z-image-turbo-mnn "Model files" interface):
+ *   d_latent fp32 [batch, in_ch, lat_h, lat_w] (lat_h, lat_w even)
+ *   d_t      fp32 [batch] model timestep, 1 = clean (pass 1 - sigma')
+ *   d_txt    bf16 [batch, s_txt, cap_dim] text features
+ *   d_out    fp32 [batch, in_ch, lat_h, lat_w] raw model output (not negated)
+ * Sequence per batch element: [(lat_h/2)(lat_w/2) image tokens; s_txt text tokens],
+ * image tokens refined by the noise refiners, text tokens by the context
+ * refiners, then all tokens through the main blocks and image tokens through
+ * the final layer.  s_txt >= 1; no padding is added (pad tokens unused). */
+ZI_API int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
+                     const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, void* d_ws,
+                     size_t ws_bytes, zi_stream_t stream);
+
+/* FlowMatch-Euler step in place (z-image-turbo-mnn "Scheduler"):
+ *   y = d_out_uncond ? d_out_uncond + guidance (d_out_cond - d_out_uncond) : d_out_cond
+ *   d_x += (sigma_next - sigma) * (-y)          (n fp32 elements)
+ * d_out_uncond may be NULL (no CFG; guidance ignored). */
+ZI_API int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond, float guidance, double sigma,
+                  double sigma_next, size_t n, zi_stream_t stream);
+
+/* Host helper: the n_steps + 1 shifted sigmas, sigma'_i = shift s / (1 + (shift-1) s)
+ * for s = linspace(1, 1/n_steps, n_steps), then 0 (z-image-turbo-mnn "Scheduler";
+ * FastVideo handoff "Scheduler").  h_sigmas has n_steps + 1 entries. */
+ZI_API int zi_sigmas(int n_steps, double shift, double* h_sigmas);
+
+/* ---------------------------------------------------------------- single steps
+ * The steps zi_block_forward / zi_model_forward chain, exposed for testing and
+ * for callers that schedule the pieces themselves. */
+
+/* Position ids of one sequence [image; text] (3-axis RoPE, ostris "Architecture";
+ * the id scheme is a reading): image token (r, c) of a grid_h x grid_w grid
+ * -> (s_txt + 1, r, c); text token j -> (j + 1, 0, 0).  d_pos int32 [grid_h*grid_w + s_txt, 3]. */
+ZI_API int zi_positions(int s_txt, int grid_h, int grid_w, int32_t* d_pos, zi_stream_t stream);
+
+/* RoPE table for n tokens: d_cos_sin fp32 [n, head_dim/2, 2] holding (cos, sin) of
+ * pos[axis] * theta^(-2j/d_axis) for rotation pair j (pairs of axis 0 first). */
+ZI_API int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, float* d_cos_sin, zi_stream_t stream);
+
+/* C[M, N] = A[M, K] B[N, K]^T, bf16 in, fp32 accumulate, bf16 out (tcgen05).
+ * K % 64 == 0, N % 256 == 0, M >= 1; rows are contiguous (strides K and N). */
+ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, zi_stream_t stream);
+
+/* Non-causal softmax(q k^T / sqrt(128)) v per head over seq tokens per batch element.
+ * d_qkv bf16 [batch*seq, 3*heads*128] (q | k | v, head h at columns h*128 of each);
+ * d_out bf16 [batch*seq, heads*128]. */
+ZI_API int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads, zi_stream_t stream);
+
+/* ---------------------------------------------------------------- device status */
+
+/* Reads (synchronously) the device error word of the current device: ZI_OK, or
+ * ZI_ERR_TIMEOUT if a kernel's bounded pipeline wait ran out since the last
+ * zi_clear_device_status(); *h_code (may be NULL) receives the raw code. */
+ZI_API int zi_device_status(int* h_code);
+
+/* Clears the device error word (synchronously).  While it is set, every
+ * pipeline kernel of the library exits at once without touching memory. */
+ZI_API int zi_clear_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZIMAGE_DIT_H */

@@ -1,0 +1,149 @@
+"""ctypes binding of libzimage_dit.so (argument marshalling only).
+
+Every function here forwards to the C entry point of the same name declared in
+include/zimage_dit.h; a non-zero status raises ZiError.  There is no fallback:
+if the shared library is missing or a call fails, the error propagates.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int, c_size_t, c_void_p
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzimage_dit.so")
+
+ZI_OK, ZI_ERR_ARG, ZI_ERR_SHAPE, ZI_ERR_ALIGN, ZI_ERR_WORKSPACE, ZI_ERR_CUDA, ZI_ERR_TIMEOUT, ZI_ERR_DEVICE = (
+    0, -1, -2, -3, -4, -5, -6, -7)
+
+
+class ZiError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: {text} (status {status})")
+        self.status = status
+
+
+class ZiConfig(ctypes.Structure):
+    _fields_ = [
+        ("dim", c_int), ("heads", c_int), ("head_dim", c_int), ("ffn", c_int), ("cap_dim", c_int),
+        ("t_freq", c_int), ("t_mid", c_int), ("in_ch", c_int), ("patch", c_int),
+        ("n_noise", c_int), ("n_ctx", c_int), ("n_main", c_int), ("rope_axes", c_int * 3),
+        ("rope_theta", c_float), ("norm_eps", c_float), ("final_eps", c_float), ("t_scale", c_float),
+    ]
+
+
+BLOCK_FIELDS = ("w_qkv", "w_out", "w13", "w2", "g_attn1", "g_attn2", "g_ffn1", "g_ffn2", "g_q", "g_k",
+                "w_ada", "b_ada")
+
+
+class ZiBlockWeights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in BLOCK_FIELDS]
+
+
+MODEL_FIELDS = ("x_emb_w", "x_emb_b", "cap_norm", "cap_w", "cap_b", "t_w1", "t_b1", "t_w2", "t_b2",
+                "final_ada_w", "final_ada_b", "final_w", "final_b")
+
+
+class ZiModelWeights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in MODEL_FIELDS] + [
+        ("noise", POINTER(ZiBlockWeights)), ("ctx", POINTER(ZiBlockWeights)), ("main", POINTER(ZiBlockWeights))]
+
+
+_SIGS = {
+    "zi_status_string": (c_char_p, [c_int]),
+    "zi_version": (c_int, []),
+    "zi_config_default": (c_int, [POINTER(ZiConfig)]),
+    "zi_ffn_padded": (c_int, [c_int]),
+    "zi_pack_qkv": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p]),
+    "zi_pack_ffn": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "zi_block_workspace_size": (c_int, [POINTER(ZiConfig), c_int, c_int, POINTER(c_size_t)]),
+    "zi_model_workspace_size": (c_int, [POINTER(ZiConfig), c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
+    "zi_block_forward": (c_int, [POINTER(ZiConfig), POINTER(ZiBlockWeights), c_void_p, c_void_p, c_int, c_int,
+                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "zi_model_forward": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
+                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "zi_euler_step": (c_int, [c_void_p, c_void_p, c_void_p, c_float, c_double, c_double, c_size_t, c_void_p]),
+    "zi_sigmas": (c_int, [c_int, c_double, POINTER(c_double)]),
+    "zi_positions": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),
+    "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
+    "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_device_status": (c_int, [POINTER(c_int)]),
+    "zi_clear_device_status": (c_int, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m stream_diffusion_transformer_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().zi_status_string(status).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != ZI_OK:
+        raise ZiError(fn, status, status_string(status))
+
+
+def call(fn: str, *args) -> None:
+    """Call a status-returning entry point and raise on error."""
+    _check(fn, getattr(lib(), fn)(*args))
+
+
+def config_default() -> ZiConfig:
+    c = ZiConfig()
+    call("zi_config_default", ctypes.byref(c))
+    return c
+
+
+def ffn_padded(ffn: int) -> int:
+    return lib().zi_ffn_padded(ffn)
+
+
+def block_workspace_size(cfg: ZiConfig, batch: int, seq: int) -> int:
+    n = c_size_t(0)
+    call("zi_block_workspace_size", ctypes.byref(cfg), batch, seq, ctypes.byref(n))
+    return n.value
+
+
+def model_workspace_size(cfg: ZiConfig, batch: int, lat_h: int, lat_w: int, s_txt: int) -> int:
+    n = c_size_t(0)
+    call("zi_model_workspace_size", ctypes.byref(cfg), batch, lat_h, lat_w, s_txt, ctypes.byref(n))
+    return n.value
+
+
+def sigmas(n_steps: int, shift: float = 3.0):
+    out = (c_double * (n_steps + 1))()
+    call("zi_sigmas", n_steps, shift, out)
+    return list(out)
+
+
+def device_status() -> int:
+    code = c_int(0)
+    st = lib().zi_device_status(ctypes.byref(code))
+    if st not in (ZI_OK, ZI_ERR_TIMEOUT):
+        _check("zi_device_status", st)
+    return code.value
+
+
+def clear_device_status() -> None:
+    call("zi_clear_device_status")
+
+
+def exported_symbols():
+    """Names of every entry point this binding declares."""
+    return list(_SIGS)

@@ -1,0 +1,348 @@
+// Persistent bf16 GEMM for sm_100a with fused epilogues:  C[M, N] = A[M, K] * B[N, K]^T.
+//
+// A is the activation (row-major, K contiguous); B is a weight in the
+// checkpoint's own [out, in] orientation, which is exactly the K-major operand
+// tcgen05 wants, so weights are used as stored.
+//
+// One CTA per SM, 6 warps:
+//   warp 0      TMA producer: 128 x 64 A tile + BN x 64 B tile per stage,
+//               128-byte swizzle, STAGES-deep mbarrier ring
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//               (M = 128, N = BN, K = 16 per instruction; fp32 accumulator in TMEM)
+//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> fused math -> global
+// The accumulator is double-buffered in TMEM (2 x BN columns), so the epilogue
+// of tile i overlaps the main loop of tile i + 1.  Tiles are walked M-fastest
+// so that CTAs running at the same time share weight tiles through L2.
+#pragma once
+#include "zi_common.cuh"
+
+namespace zi {
+
+// Maps a global row of the token buffer to its batch element and to its index
+// in one sequence's position table.  Rows [0, n_a) hold segment A (len_a rows
+// per batch element), rows [n_a, ...) hold segment B (len_b rows per element);
+// in a sequence, segment A occupies positions [0, len_a) and B [len_a, len_a + len_b).
+struct RowMap {
+  int n_a, len_a, len_b;
+  ZI_DEV int batch(int r) const { return r < n_a ? r / len_a : (r - n_a) / len_b; }
+  ZI_DEV int pos(int r) const { return r < n_a ? r % len_a : len_a + (r - n_a) % len_b; }
+};
+
+enum EpiKind : int {
+  EPI_BF16 = 0,     // out bf16 [M, ldo]
+  EPI_F32_BIAS = 1, // out fp32 [M, ldo] = acc + bias
+  EPI_QKV = 2,      // q, k: RMSNorm over each 128-wide head, gain, RoPE; v: plain; out bf16 [M, 3D]
+  EPI_SWIGLU = 3,   // 256-wide tile = 128 gate + 128 up columns -> out bf16 SiLU(gate) * up [M, N/2]
+  EPI_UNPATCH = 4,  // final linear: acc + bias scattered to the latent [B, C, H, W] fp32
+};
+
+struct EpiParams {
+  void* out;
+  int ldo;                 // row stride of `out` in elements
+  const uint16_t* bias;    // bf16 [N] (EPI_F32_BIAS, EPI_UNPATCH)
+  const float2* rope;      // (cos, sin) [n_pos][head_dim / 2] (EPI_QKV)
+  const uint16_t* g_q;     // bf16 [128] QK-RMSNorm gains (EPI_QKV)
+  const uint16_t* g_k;
+  float eps;
+  int dim;                 // D: column offset of k in the fused projection (EPI_QKV)
+  int row_off;             // global row of local row 0 (for RowMap)
+  RowMap map;
+  int s_img, grid_w, lat_c, lat_h, lat_w;  // EPI_UNPATCH
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr uint32_t kABytes = 128u * 64u * 2u;
+  static constexpr uint32_t kBBytes = uint32_t(BN) * 64u * 2u;
+  static constexpr uint32_t kStage = kABytes + kBBytes;
+  static constexpr uint32_t kBarOff = STAGES * kStage;
+  static constexpr uint32_t kBytes = kBarOff + 256u + 1024u;  // + barriers + alignment slack
+  static constexpr uint32_t kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                        : (2 * BN <= 256) ? 256 : 512;
+};
+
+// Store 32 fp32 values as bf16 (64 contiguous bytes).
+ZI_DEV void store_bf16x32(uint16_t* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = w;
+  }
+}
+
+template <int EPI, int BN>
+ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const EpiParams& ep) {
+  uint32_t v[32];
+  float f[32];
+  if constexpr (EPI == EPI_BF16 || EPI == EPI_F32_BIAS) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      tmem_ld32_sync(tbase + c * 32, v);
+      if (row_ok) {
+        const int col = n0 + c * 32;
+        if constexpr (EPI == EPI_BF16) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+          store_bf16x32(static_cast<uint16_t*>(ep.out) + size_t(row) * ep.ldo + col, f);
+        } else {
+          float4* d = reinterpret_cast<float4*>(static_cast<float*>(ep.out) + size_t(row) * ep.ldo + col);
+          const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + col);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 b = __ldg(bp + q);
+            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float4 o;
+              o.x = __uint_as_float(v[8 * q + 4 * h + 0]) + bf16_to_f32(uint16_t(bw[2 * h] & 0xFFFF));
+              o.y = __uint_as_float(v[8 * q + 4 * h + 1]) + bf16_to_f32(uint16_t(bw[2 * h] >> 16));
+              o.z = __uint_as_float(v[8 * q + 4 * h + 2]) + bf16_to_f32(uint16_t(bw[2 * h + 1] & 0xFFFF));
+              o.w = __uint_as_float(v[8 * q + 4 * h + 3]) + bf16_to_f32(uint16_t(bw[2 * h + 1] >> 16));
+              d[2 * q + h] = o;
+            }
+          }
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_QKV) {
+    static_assert(BN == 256, "QKV epilogue works on two 128-wide heads per tile");
+    const int region = n0 / ep.dim;  // 0 = q, 1 = k, 2 = v
+    uint16_t* orow = static_cast<uint16_t*>(ep.out) + size_t(row) * ep.ldo;
+    if (region == 2) {
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        tmem_ld32_sync(tbase + c * 32, v);
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+          store_bf16x32(orow + n0 + c * 32, f);
+        }
+      }
+      return;
+    }
+    const uint16_t* g = region == 0 ? ep.g_q : ep.g_k;
+    const int p = row_ok ? ep.map.pos(row + ep.row_off) : 0;
+    const float2* rp = ep.rope + size_t(p) * 64;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32_sync(tbase + hh * 128 + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x = __uint_as_float(v[i]);
+          ss = fmaf(x, x, ss);
+        }
+      }
+      const float r = rsqrtf(ss * (1.0f / 128.0f) + ep.eps);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32_sync(tbase + hh * 128 + c * 32, v);
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int d0 = c * 32 + 2 * i;
+            const float a = __uint_as_float(v[2 * i]) * r * bf16_to_f32(__ldg(g + d0));
+            const float b = __uint_as_float(v[2 * i + 1]) * r * bf16_to_f32(__ldg(g + d0 + 1));
+            const float2 cs = __ldg(rp + c * 16 + i);
+            f[2 * i] = a * cs.x - b * cs.y;
+            f[2 * i + 1] = a * cs.y + b * cs.x;
+          }
+          store_bf16x32(orow + n0 + hh * 128 + c * 32, f);
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    static_assert(BN == 256, "SwiGLU epilogue pairs 128 gate with 128 up columns");
+    uint32_t u[32];
+    uint16_t* orow = static_cast<uint16_t*>(ep.out) + size_t(row) * ep.ldo + n0 / 2;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld32(tbase + c * 32, v);
+      tmem_ld32(tbase + 128 + c * 32, u);
+      tmem_wait_ld();
+      reg_fence32(v);
+      reg_fence32(u);
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float gt = __uint_as_float(v[i]);
+          const float up = __uint_as_float(u[i]);
+          f[i] = gt / (1.0f + __expf(-gt)) * up;
+        }
+        store_bf16x32(orow + c * 32, f);
+      }
+    }
+  } else if constexpr (EPI == EPI_UNPATCH) {
+    float* out = static_cast<float*>(ep.out);
+    const int gr = row_ok ? row + ep.row_off : 0;
+    const int b = gr / ep.s_img, t = gr % ep.s_img;
+    const int ty = t / ep.grid_w, tx = t % ep.grid_w;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      tmem_ld32_sync(tbase + c * 32, v);
+      if (row_ok) {
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+          const int feat = n0 + c * 32 + i;
+          const int ch = feat % ep.lat_c, pq = feat / ep.lat_c;
+          const int y = 2 * ty + (pq >> 1), x = 2 * tx + (pq & 1);
+          out[((size_t(b) * ep.lat_c + ch) * ep.lat_h + y) * ep.lat_w + x] =
+              __uint_as_float(v[i]) + bf16_to_f32(__ldg(ep.bias + feat));
+        }
+      }
+    }
+  }
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                        int N, int K, EpiParams ep) {
+  using L = GemmSmem<BN, STAGES>;
+  constexpr int BM = 128, BK = 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (device_error_set()) return;  // an earlier kernel timed out: leave everything untouched
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (M + BM - 1) / BM;
+  const int num_tiles = num_m * (N / BN);
+  const int KB = K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * L::kStage;
+          mbar_arrive_expect_tx(&full[s], L::kStage);
+          tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
+          tma_load_2d(sa + L::kABytes, &tmB, &full[s], kb * BK, n0);
+          ++it;
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA exits.
+        const uint32_t n = it < uint32_t(STAGES) ? it : uint32_t(STAGES);
+        for (uint32_t j = 1; j <= n; ++j) {
+          const uint32_t k = it - j;
+          volatile int never = 0;
+          mbar_wait(&full[k % STAGES], (k / STAGES) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t u = uint32_t(local) >> 1;
+        if (!mbar_wait(&tempty[acc], (u & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&full[s], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * L::kStage);
+          const uint32_t b_addr = a_addr + L::kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma(d, smem_desc_sw128(a_addr + k * 32, 16), smem_desc_sw128(b_addr + k * 32, 16), idesc,
+                   (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+          ++it;
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        // Wait until every MMA issued so far has finished before TMEM is freed.
+        tc_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
+      }
+    }
+  } else {
+    const int q = warp & 3;  // this warp's TMEM lane quarter
+    const int row_in_tile = q * 32 + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t u = uint32_t(local) >> 1;
+      if (!mbar_wait(&tfull[acc], u & 1u, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+      const int row = m0 + row_in_tile;
+      const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+      gemm_epilogue<EPI, BN>(tb, row, row < M, n0, ep);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace zi

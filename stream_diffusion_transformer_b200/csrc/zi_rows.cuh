@@ -1,0 +1,340 @@
+// Bandwidth-bound kernels: row norms with modulation and gated residuals,
+// positions and the RoPE table, the timestep MLP, the batched adaLN GEMV,
+// patchify, and the Euler / CFG step.  One CTA per row for the row kernels
+// (128 threads, float4 / 8-byte bf16 vectors, every byte read once).
+#pragma once
+#include "zi_common.cuh"
+#include "zi_gemm.cuh"
+
+namespace zi {
+
+constexpr int kRowThreads = 128;
+constexpr int kRowMaxVec = 8;  // float4 per thread: rows up to 128 * 8 * 4 = 4096 wide
+
+ZI_DEV float block_sum_128(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();  // `red` may still be read from a previous reduction
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  return red[0] + red[1] + red[2] + red[3];
+}
+
+ZI_DEV float4 ld_bf16x4(const uint16_t* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+ZI_DEV void st_bf16x4(uint16_t* p, float4 v) {
+  uint2 u;
+  u.x = pack_bf16x2(v.x, v.y);
+  u.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+// h[row] = bf16( gain * x / sqrt(mean(x^2) + eps) * (1 + scale[batch(row)]) )
+// x is fp32 (TIn = float) or bf16 (TIn = uint16_t); scale may be null (no modulation).
+template <typename TIn>
+__global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restrict__ x, int D,
+                                                              const uint16_t* __restrict__ gain,
+                                                              const float* __restrict__ scale, int scale_ld,
+                                                              RowMap map, int row_off, float eps,
+                                                              uint16_t* __restrict__ h) {
+  __shared__ float red[4];
+  const int row = blockIdx.x;
+  const int nvec = D >> 2;
+  float4 v[kRowMaxVec];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < nvec) {
+      if constexpr (sizeof(TIn) == 4) {
+        v[k] = reinterpret_cast<const float4*>(x + size_t(row) * D)[i];
+      } else {
+        v[k] = ld_bf16x4(reinterpret_cast<const uint16_t*>(x) + size_t(row) * D + 4 * i);
+      }
+      ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+    }
+  }
+  const float r = rsqrtf(block_sum_128(ss, red) / float(D) + eps);
+  const float* sc = scale ? scale + size_t(map.batch(row + row_off)) * scale_ld : nullptr;
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < nvec) {
+      const float4 g = ld_bf16x4(gain + 4 * i);
+      float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (sc) {
+        const float4 s = reinterpret_cast<const float4*>(sc)[i];
+        m = make_float4(1.f + s.x, 1.f + s.y, 1.f + s.z, 1.f + s.w);
+      }
+      st_bf16x4(h + size_t(row) * D + 4 * i,
+                make_float4(v[k].x * r * g.x * m.x, v[k].y * r * g.y * m.y, v[k].z * r * g.z * m.z,
+                            v[k].w * r * g.w * m.w));
+    }
+  }
+}
+
+enum NextNorm : int { NEXT_NONE = 0, NEXT_RMS = 1, NEXT_LAYERNORM = 2 };
+
+// Gated residual with the post-sublayer RMSNorm, fused with the next sublayer's
+// pre-norm:
+//   x_out = x_in + gate * g_post * o / sqrt(mean(o^2) + eps)      (gate = tanh(raw) or 1)
+//   h     = g_next * x_out / sqrt(mean(x_out^2) + eps) * (1 + scale)     (NEXT_RMS)
+//   h     = (x_out - mean) / sqrt(var + eps_ln) * (1 + scale)            (NEXT_LAYERNORM)
+// h is written only for rows < next_rows.
+struct PostParams {
+  const float* x_in;
+  float* x_out;
+  const uint16_t* o;
+  const uint16_t* g_post;
+  const float* gate;  // raw adaLN gate [B][gate_ld] or null (gate = 1)
+  int gate_ld;
+  int next;
+  const uint16_t* g_next;  // NEXT_RMS gain
+  const float* scale;      // [B][scale_ld] or null (no modulation)
+  int scale_ld;
+  int next_rows;
+  uint16_t* h;
+  RowMap map;
+  int row_off;  // global row of local row 0 (for the batch lookup)
+  int D;
+  float eps, eps_ln;
+};
+
+__global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p) {
+  __shared__ float red[4];
+  const int row = blockIdx.x;
+  const int D = p.D, nvec = D >> 2;
+  const int b = p.map.batch(row + p.row_off);
+  float4 v[kRowMaxVec];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < nvec) {
+      v[k] = ld_bf16x4(p.o + size_t(row) * D + 4 * i);
+      ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+    }
+  }
+  const float ro = rsqrtf(block_sum_128(ss, red) / float(D) + p.eps);
+  const float* gt = p.gate ? p.gate + size_t(b) * p.gate_ld : nullptr;
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < nvec) {
+      const float4 x = reinterpret_cast<const float4*>(p.x_in + size_t(row) * D)[i];
+      const float4 g = ld_bf16x4(p.g_post + 4 * i);
+      float4 a = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (gt) {
+        const float4 r = reinterpret_cast<const float4*>(gt)[i];
+        a = make_float4(tanhf(r.x), tanhf(r.y), tanhf(r.z), tanhf(r.w));
+      }
+      float4 y;
+      y.x = x.x + a.x * g.x * (v[k].x * ro);
+      y.y = x.y + a.y * g.y * (v[k].y * ro);
+      y.z = x.z + a.z * g.z * (v[k].z * ro);
+      y.w = x.w + a.w * g.w * (v[k].w * ro);
+      reinterpret_cast<float4*>(p.x_out + size_t(row) * D)[i] = y;
+      v[k] = y;
+      s1 += y.x + y.y + y.z + y.w;
+      s2 += y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
+    }
+  }
+  if (p.next == NEXT_NONE || row >= p.next_rows) return;
+  float mu = 0.f, r;
+  if (p.next == NEXT_RMS) {
+    r = rsqrtf(block_sum_128(s2, red) / float(D) + p.eps);
+  } else {
+    mu = block_sum_128(s1, red) / float(D);
+    // variance from the centred values (second pass over registers)
+    float sc = 0.f;
+#pragma unroll
+    for (int k = 0; k < kRowMaxVec; ++k) {
+      const int i = threadIdx.x + k * kRowThreads;
+      if (i < nvec) {
+        const float a = v[k].x - mu, bq = v[k].y - mu, c = v[k].z - mu, d = v[k].w - mu;
+        sc += a * a + bq * bq + c * c + d * d;
+      }
+    }
+    r = rsqrtf(block_sum_128(sc, red) / float(D) + p.eps_ln);
+  }
+  const float* sc = p.scale ? p.scale + size_t(b) * p.scale_ld : nullptr;
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < nvec) {
+      float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (p.next == NEXT_RMS) g = ld_bf16x4(p.g_next + 4 * i);
+      float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (sc) {
+        const float4 s = reinterpret_cast<const float4*>(sc)[i];
+        m = make_float4(1.f + s.x, 1.f + s.y, 1.f + s.z, 1.f + s.w);
+      }
+      st_bf16x4(p.h + size_t(row) * D + 4 * i,
+                make_float4((v[k].x - mu) * r * g.x * m.x, (v[k].y - mu) * r * g.y * m.y,
+                            (v[k].z - mu) * r * g.z * m.z, (v[k].w - mu) * r * g.w * m.w));
+    }
+  }
+}
+
+// Position ids of one sequence [image tokens; text tokens]:
+// image token (r, c) -> (s_txt + 1, r, c); text token j -> (j + 1, 0, 0).
+__global__ void positions_kernel(int s_txt, int grid_h, int grid_w, int* __restrict__ pos) {
+  const int n_img = grid_h * grid_w;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n_img + s_txt) return;
+  int a, b, c;
+  if (t < n_img) {
+    a = s_txt + 1;
+    b = t / grid_w;
+    c = t % grid_w;
+  } else {
+    a = t - n_img + 1;
+    b = 0;
+    c = 0;
+  }
+  pos[3 * t + 0] = a;
+  pos[3 * t + 1] = b;
+  pos[3 * t + 2] = c;
+}
+
+// (cos, sin) of pos[axis] * theta^(-2j/d_axis) for every token and rotation
+// pair; pairs [0, a0/2) use axis 0, the next a1/2 axis 1, the last a2/2 axis 2.
+// Angles are formed in fp64 and rounded to fp32 once.
+__global__ void rope_table_kernel(const int* __restrict__ pos, int n, int a0, int a1, int a2, double theta,
+                                  float2* __restrict__ out) {
+  const int pairs = (a0 + a1 + a2) / 2;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * pairs) return;
+  const int t = idx / pairs, j = idx % pairs;
+  int axis, jj, da;
+  if (j < a0 / 2) {
+    axis = 0; jj = j; da = a0;
+  } else if (j < (a0 + a1) / 2) {
+    axis = 1; jj = j - a0 / 2; da = a1;
+  } else {
+    axis = 2; jj = j - (a0 + a1) / 2; da = a2;
+  }
+  const double omega = pow(theta, -2.0 * double(jj) / double(da));
+  const double ang = double(pos[3 * t + axis]) * omega;
+  double s, c;
+  sincos(ang, &s, &c);
+  out[idx] = make_float2(float(c), float(s));
+}
+
+// Timestep conditioning for one batch element per CTA (256 threads):
+// e = [cos(1000 t f_k), sin(1000 t f_k)], f_k = 10000^(-k/128) (sinusoid in fp64);
+// c = W2 SiLU(W1 e + b1) + b2; also writes SiLU(c) for the final layer's adaLN.
+__global__ void __launch_bounds__(256) timestep_mlp_kernel(const float* __restrict__ t, float t_scale, int t_freq,
+                                                           int t_mid, int ada, const uint16_t* __restrict__ w1,
+                                                           const uint16_t* __restrict__ b1,
+                                                           const uint16_t* __restrict__ w2,
+                                                           const uint16_t* __restrict__ b2, float* __restrict__ c,
+                                                           float* __restrict__ silu_c) {
+  extern __shared__ float sh[];
+  float* e = sh;            // [t_freq]
+  float* hid = sh + t_freq; // [t_mid]
+  const int b = blockIdx.x;
+  const int half = t_freq / 2;
+  const double tin = double(t[b]) * double(t_scale);
+  for (int k = threadIdx.x; k < half; k += blockDim.x) {
+    const double f = exp(-log(10000.0) * double(k) / double(half));
+    double s, co;
+    sincos(tin * f, &s, &co);
+    e[k] = float(co);
+    e[k + half] = float(s);
+  }
+  __syncthreads();
+  for (int o = threadIdx.x; o < t_mid; o += blockDim.x) {
+    float acc = bf16_to_f32(b1[o]);
+    const uint16_t* wr = w1 + size_t(o) * t_freq;
+    for (int i = 0; i < t_freq; ++i) acc = fmaf(bf16_to_f32(wr[i]), e[i], acc);
+    hid[o] = acc / (1.0f + expf(-acc));
+  }
+  __syncthreads();
+  for (int o = threadIdx.x; o < ada; o += blockDim.x) {
+    float acc = bf16_to_f32(b2[o]);
+    const uint16_t* wr = w2 + size_t(o) * t_mid;
+    for (int i = 0; i < t_mid; ++i) acc = fmaf(bf16_to_f32(wr[i]), hid[i], acc);
+    c[size_t(b) * ada + o] = acc;
+    silu_c[size_t(b) * ada + o] = acc / (1.0f + expf(-acc));
+  }
+}
+
+// All adaLN projections of a forward in one launch: segment s maps its input
+// vector (c, or SiLU(c) for the final layer) through w_s [rows_s, 256] + b_s into
+// out[b][off_s + row].  One warp per output row, 16-byte weight loads.
+constexpr int kMaxAdaSegs = 40;
+struct AdaSegs {
+  const uint16_t* w[kMaxAdaSegs];
+  const uint16_t* b[kMaxAdaSegs];
+  int rows[kMaxAdaSegs];
+  int off[kMaxAdaSegs];
+  int silu[kMaxAdaSegs];
+  int n;
+};
+
+__global__ void __launch_bounds__(256) ada_gemv_kernel(AdaSegs segs, const float* __restrict__ c,
+                                                       const float* __restrict__ silu_c, int batch, int out_ld,
+                                                       float* __restrict__ out) {
+  // ada width fixed at 256: each lane owns 8 consecutive inputs.
+  const int s = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows = segs.rows[s];
+  const float* in = segs.silu[s] ? silu_c : c;
+  for (int r = blockIdx.x * 8 + warp; r < rows; r += gridDim.x * 8) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(segs.w[s] + size_t(r) * 256 + lane * 8);
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+    float wf[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      wf[2 * q] = __uint_as_float(ww[q] << 16);
+      wf[2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
+    }
+    const float bias = bf16_to_f32(segs.b[s][r]);
+    for (int b = 0; b < batch; ++b) {
+      const float4 i0 = *reinterpret_cast<const float4*>(in + size_t(b) * 256 + lane * 8);
+      const float4 i1 = *reinterpret_cast<const float4*>(in + size_t(b) * 256 + lane * 8 + 4);
+      float acc = wf[0] * i0.x + wf[1] * i0.y + wf[2] * i0.z + wf[3] * i0.w + wf[4] * i1.x + wf[5] * i1.y +
+                  wf[6] * i1.z + wf[7] * i1.w;
+      acc = warp_sum(acc);
+      if (lane == 0) out[size_t(b) * out_ld + segs.off[s] + r] = acc + bias;
+    }
+  }
+}
+
+// latent [B, C, H, W] fp32 -> tokens [B * (H/2)(W/2), 4C] bf16, feature (i*2 + j)*C + c.
+__global__ void patchify_kernel(const float* __restrict__ lat, int B, int C, int H, int W,
+                                uint16_t* __restrict__ tok) {
+  const int gw = W / 2, gh = H / 2, F = 4 * C;
+  const size_t total = size_t(B) * gh * gw * F;
+  const size_t idx = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int f = int(idx % F);
+  const size_t tkn = idx / F;
+  const int b = int(tkn / (size_t(gh) * gw));
+  const int t = int(tkn % (size_t(gh) * gw));
+  const int r = t / gw, s = t % gw;
+  const int c = f % C, pq = f / C;
+  const float v = lat[((size_t(b) * C + c) * H + 2 * r + (pq >> 1)) * W + 2 * s + (pq & 1)];
+  __nv_bfloat16 hb = __float2bfloat16_rn(v);
+  tok[idx] = *reinterpret_cast<uint16_t*>(&hb);
+}
+
+// x += (sigma_next - sigma) * (-y),  y = out_u + g (out_c - out_u)  (or out_c without CFG).
+__global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ oc, const float* __restrict__ ou,
+                             float g, float dt, size_t n) {
+  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float y = oc[i];
+  if (ou) y = ou[i] + g * (y - ou[i]);
+  x[i] = x[i] + dt * (-y);
+}
+
+}  // namespace zi

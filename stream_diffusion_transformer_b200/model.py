@@ -1,0 +1,216 @@
+"""Python front end of the C ABI: device-resident weights, workspaces and calls.
+
+PyTorch is used only to own device memory and streams; every step of the
+forward runs in libzimage_dit.so.  bf16 tensors are handed over as raw bits.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Callable, Dict, Iterable, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import abi
+
+Bits = np.ndarray  # uint16 bf16 bit patterns
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def upload_bits(bits: Bits, device) -> torch.Tensor:
+    """bf16 bit patterns (uint16 numpy) -> a bf16 tensor on `device`."""
+    host = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return host.to(device).view(torch.bfloat16)
+
+
+def make_config(dims) -> abi.ZiConfig:
+    """ZiConfig from any object with the model's size attributes (dim, heads, ...)."""
+    c = abi.config_default()
+    for name in ("dim", "heads", "head_dim", "ffn", "cap_dim", "t_freq", "t_mid", "in_ch", "patch",
+                 "n_noise", "n_ctx", "n_main"):
+        setattr(c, name, int(getattr(dims, name)))
+    axes = getattr(dims, "rope_axes", (32, 48, 48))
+    for i in range(3):
+        c.rope_axes[i] = int(axes[i])
+    return c
+
+
+def block_keys(prefix: str, modulated: bool) -> List[str]:
+    a = f"{prefix}.attention"
+    k = [f"{a}.to_q.weight", f"{a}.to_k.weight", f"{a}.to_v.weight", f"{a}.to_out.weight",
+         f"{a}.norm_q.weight", f"{a}.norm_k.weight", f"{prefix}.attention_norm1.weight",
+         f"{prefix}.attention_norm2.weight", f"{prefix}.ffn_norm1.weight", f"{prefix}.ffn_norm2.weight",
+         f"{prefix}.feed_forward.w1.weight", f"{prefix}.feed_forward.w2.weight", f"{prefix}.feed_forward.w3.weight"]
+    if modulated:
+        k += [f"{prefix}.adaLN_modulation.weight", f"{prefix}.adaLN_modulation.bias"]
+    return k
+
+
+TOP_KEYS = {
+    "x_emb_w": "x_embedder.weight", "x_emb_b": "x_embedder.bias",
+    "cap_norm": "cap_embedder.norm.weight", "cap_w": "cap_embedder.linear.weight",
+    "cap_b": "cap_embedder.linear.bias",
+    "t_w1": "t_embedder.linear1.weight", "t_b1": "t_embedder.linear1.bias",
+    "t_w2": "t_embedder.linear2.weight", "t_b2": "t_embedder.linear2.bias",
+    "final_ada_w": "final_layer.adaLN_modulation.weight", "final_ada_b": "final_layer.adaLN_modulation.bias",
+    "final_w": "final_layer.linear.weight", "final_b": "final_layer.linear.bias",
+}
+
+
+class DeviceBlock:
+    """One block's weights in the library's layout (fused qkv, interleaved w13, padded w2)."""
+
+    def __init__(self, cfg: abi.ZiConfig, prefix: str, bits: Dict[str, Bits], modulated: bool, device):
+        D, F = cfg.dim, cfg.ffn
+        Fp = abi.ffn_padded(F)
+        a = f"{prefix}.attention"
+        self.t: Dict[str, torch.Tensor] = {}
+        w_qkv = torch.empty((3 * D, D), dtype=torch.bfloat16, device=device)
+        for i, nm in enumerate(("to_q", "to_k", "to_v")):
+            w_qkv[i * D:(i + 1) * D].copy_(upload_bits(bits[f"{a}.{nm}.weight"], "cpu"))
+        self.t["w_qkv"] = w_qkv
+        self.t["w_out"] = upload_bits(bits[f"{a}.to_out.weight"], device)
+        ff = f"{prefix}.feed_forward"
+        w1 = upload_bits(bits[f"{ff}.w1.weight"], device)
+        w3 = upload_bits(bits[f"{ff}.w3.weight"], device)
+        w2 = upload_bits(bits[f"{ff}.w2.weight"], device)
+        self.t["w13"] = torch.empty((2 * Fp, D), dtype=torch.bfloat16, device=device)
+        self.t["w2"] = torch.empty((D, Fp), dtype=torch.bfloat16, device=device)
+        abi.call("zi_pack_ffn", _p(w1), _p(w3), _p(w2), F, D, _p(self.t["w13"]), _p(self.t["w2"]), _stream())
+        torch.cuda.current_stream().synchronize()  # the temporaries w1, w3, w2 are freed on return
+        for fld, key in (("g_attn1", f"{prefix}.attention_norm1.weight"),
+                         ("g_attn2", f"{prefix}.attention_norm2.weight"),
+                         ("g_ffn1", f"{prefix}.ffn_norm1.weight"), ("g_ffn2", f"{prefix}.ffn_norm2.weight"),
+                         ("g_q", f"{a}.norm_q.weight"), ("g_k", f"{a}.norm_k.weight")):
+            self.t[fld] = upload_bits(bits[key], device)
+        if modulated:
+            self.t["w_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.weight"], device)
+            self.t["b_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.bias"], device)
+        self.modulated = modulated
+        self.struct = abi.ZiBlockWeights(**{f: (self.t[f].data_ptr() if f in self.t else None)
+                                            for f in abi.BLOCK_FIELDS})
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self.t.values())
+
+
+class DiT:
+    """The S3-DiT transformer on one GPU, weights resident in HBM."""
+
+    def __init__(self, cfg: abi.ZiConfig, fetch: Callable[[Sequence[str]], Dict[str, Bits]], device="cuda"):
+        """fetch(keys) -> {key: bf16 bits} is called once per block and once for the rest,
+        so a 12 GB model never has to sit in host memory at once."""
+        self.cfg = cfg
+        self.device = torch.device(device)
+        abi.lib()
+        top = fetch(list(TOP_KEYS.values()))
+        self.top = {f: upload_bits(top[k], self.device) for f, k in TOP_KEYS.items()}
+        self.noise = [DeviceBlock(cfg, f"noise_refiner.{i}", fetch(block_keys(f"noise_refiner.{i}", True)), True,
+                                  self.device) for i in range(cfg.n_noise)]
+        self.ctx = [DeviceBlock(cfg, f"context_refiner.{i}", fetch(block_keys(f"context_refiner.{i}", False)),
+                                False, self.device) for i in range(cfg.n_ctx)]
+        self.main = [DeviceBlock(cfg, f"layers.{i}", fetch(block_keys(f"layers.{i}", True)), True, self.device)
+                     for i in range(cfg.n_main)]
+        self._noise_arr = (abi.ZiBlockWeights * max(1, len(self.noise)))(*[b.struct for b in self.noise])
+        self._ctx_arr = (abi.ZiBlockWeights * max(1, len(self.ctx)))(*[b.struct for b in self.ctx])
+        self._main_arr = (abi.ZiBlockWeights * len(self.main))(*[b.struct for b in self.main])
+        kw = {f: self.top[f].data_ptr() for f in abi.MODEL_FIELDS}
+        self.weights = abi.ZiModelWeights(**kw)
+        self.weights.noise = ctypes.cast(self._noise_arr, ctypes.POINTER(abi.ZiBlockWeights))
+        self.weights.ctx = ctypes.cast(self._ctx_arr, ctypes.POINTER(abi.ZiBlockWeights))
+        self.weights.main = ctypes.cast(self._main_arr, ctypes.POINTER(abi.ZiBlockWeights))
+        self._ws: Dict[tuple, torch.Tensor] = {}
+
+    def nbytes(self) -> int:
+        n = sum(t.numel() * t.element_size() for t in self.top.values())
+        return n + sum(b.nbytes() for b in self.noise + self.ctx + self.main)
+
+    def workspace(self, batch: int, lat_h: int, lat_w: int, s_txt: int) -> torch.Tensor:
+        key = (batch, lat_h, lat_w, s_txt)
+        if key not in self._ws:
+            n = abi.model_workspace_size(self.cfg, batch, lat_h, lat_w, s_txt)
+            self._ws[key] = torch.empty(n, dtype=torch.uint8, device=self.device)
+        return self._ws[key]
+
+    def forward(self, latent: torch.Tensor, t: torch.Tensor, txt: torch.Tensor,
+                out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """latent fp32 [B, C, H/8, W/8], t fp32 [B] (1 = clean), txt bf16 [B, L, cap_dim] -> raw output."""
+        B, C, Hl, Wl = latent.shape
+        L = txt.shape[1]
+        assert latent.dtype == torch.float32 and t.dtype == torch.float32 and txt.dtype == torch.bfloat16
+        assert latent.is_contiguous() and txt.is_contiguous() and t.is_contiguous()
+        if out is None:
+            out = torch.empty_like(latent)
+        ws = self.workspace(B, Hl, Wl, L)
+        abi.call("zi_model_forward", ctypes.byref(self.cfg), ctypes.byref(self.weights), B, Hl, Wl, L,
+                 _p(latent), _p(t), _p(txt), _p(out), _p(ws), ws.numel(), _stream(stream))
+        return out
+
+
+def block_forward(cfg: abi.ZiConfig, blk: DeviceBlock, c: Optional[torch.Tensor], pos: torch.Tensor,
+                  x_in: torch.Tensor, x_out: Optional[torch.Tensor] = None,
+                  ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One block on x_in fp32 [B, S, D]; pos int32 [S, 3]; c fp32 [B, 256] (or None if unmodulated)."""
+    B, S, D = x_in.shape
+    if x_out is None:
+        x_out = torch.empty_like(x_in)
+    need = abi.block_workspace_size(cfg, B, S)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=x_in.device)
+    abi.call("zi_block_forward", ctypes.byref(cfg), ctypes.byref(blk.struct), _p(c), _p(pos), B, S,
+             _p(x_in), _p(x_out), _p(ws), ws.numel(), _stream())
+    return x_out
+
+
+# ------------------------------------------------------------------ single steps
+
+def positions(s_txt: int, grid_h: int, grid_w: int, device="cuda") -> torch.Tensor:
+    pos = torch.empty((grid_h * grid_w + s_txt, 3), dtype=torch.int32, device=device)
+    abi.call("zi_positions", s_txt, grid_h, grid_w, _p(pos), _stream())
+    return pos
+
+
+def rope_table(cfg: abi.ZiConfig, pos: torch.Tensor) -> torch.Tensor:
+    out = torch.empty((pos.shape[0], cfg.head_dim // 2, 2), dtype=torch.float32, device=pos.device)
+    abi.call("zi_rope_table", ctypes.byref(cfg), _p(pos), pos.shape[0], _p(out), _stream())
+    return out
+
+
+def gemm(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """a bf16 [M, K] @ b bf16 [N, K]^T -> bf16 [M, N]."""
+    M, K = a.shape
+    N = b.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    abi.call("zi_gemm_bf16", _p(a), _p(b), _p(out), M, N, K, _stream())
+    return out
+
+
+def attention(qkv: torch.Tensor, batch: int, seq: int, heads: int,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((batch * seq, heads * 128), dtype=torch.bfloat16, device=qkv.device)
+    abi.call("zi_attention", _p(qkv), _p(out), batch, seq, heads, _stream())
+    return out
+
+
+def euler_step(x: torch.Tensor, out_cond: torch.Tensor, out_uncond: Optional[torch.Tensor], guidance: float,
+               sigma: float, sigma_next: float) -> torch.Tensor:
+    abi.call("zi_euler_step", _p(x), _p(out_cond), _p(out_uncond), float(guidance), float(sigma),
+             float(sigma_next), x.numel(), _stream())
+    return x
+
+
+def pack_qkv(wq: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor) -> torch.Tensor:
+    D = wq.shape[0]
+    out = torch.empty((3 * D, D), dtype=torch.bfloat16, device=wq.device)
+    abi.call("zi_pack_qkv", _p(wq), _p(wk), _p(wv), D, _p(out), _stream())
+    return out

@@ -1,0 +1,70 @@
+"""GPU parity of zi_block_forward against the CPU oracle's block.
+
+Bars: block output rel-L2 <= 2e-2 and cosine >= 0.999 against the oracle
+(fp64, same bf16 weights); the block's update x_out - x_in cosine >= 0.99, so
+a broken sublayer cannot hide behind the residual."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from gpu_util import assert_parity, require_gpu, torch
+import zimage_inputs as zi
+from oracle import zimage_ref as ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+    from stream_diffusion_transformer_b200 import abi
+    abi.lib()
+    abi.clear_device_status()
+    yield
+    assert abi.device_status() == 0
+
+
+def run_block(d, prefix, modulated, batch, s_txt, gh, gw, seed, in_place=False):
+    from stream_diffusion_transformer_b200 import model
+    cfg = model.make_config(d)
+    keys = model.block_keys(prefix, modulated)
+    bits = zi.make_weights(d, seed=seed, keys=keys)
+    S = gh * gw + s_txt
+    x = zi.make_stream(d, batch, S, seed=seed)
+    c = zi.make_cond(d, batch, seed=seed) if modulated else None
+    blk = model.DeviceBlock(cfg, prefix, bits, modulated, "cuda")
+    pos = model.positions(s_txt, gh, gw)
+    xt = torch.from_numpy(x).cuda()
+    ct = None if c is None else torch.from_numpy(c).cuda()
+    out = model.block_forward(cfg, blk, ct, pos, xt, xt if in_place else None)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    W = ref.Weights(bits)
+    ang = ref.rope_angles(ref.position_ids(s_txt, gh, gw), d.rope_axes)
+    for b in range(batch):
+        want = ref.block_forward(x[b].astype(np.float64), W, prefix, d, ang, None if c is None else c[b].astype(np.float64))
+        assert_parity(got[b], want, rel=2e-2, cos=0.999, what=f"{prefix} b={b}")
+        assert_parity(got[b] - x[b], want - x[b], rel=1.0, cos=0.99, what=f"{prefix} delta b={b}")
+
+
+@pytest.mark.parametrize("modulated", [True, False])
+def test_tiny_block(modulated):
+    """hidden 256 (2 heads), FFN 688 (padded to 768 inside), 64 image + 32 text tokens."""
+    run_block(zi.TINY, "layers.0", modulated, 1, 32, 8, 8, seed=1)
+
+
+def test_tiny_block_batch_ragged_in_place():
+    """batch 2, 5 x 7 image tokens + 17 text tokens: ragged query/key tiles, in-place update."""
+    run_block(zi.TINY, "layers.0", True, 2, 17, 5, 7, seed=2, in_place=True)
+
+
+def test_full_width_block_1152_tokens():
+    """One main block at full width: 512x512 image (1,024 tokens) + 128 text tokens."""
+    run_block(dataclasses.replace(zi.FULL, n_noise=0, n_ctx=0, n_main=1), "layers.0", True, 1, 128, 32, 32, seed=3)
+
+
+def test_full_width_unmodulated_text_block():
+    """A context-refiner-shaped block on 32 text tokens only (a single partial tile)."""
+    d = dataclasses.replace(zi.FULL, n_noise=0, n_ctx=1, n_main=1)
+    run_block(d, "context_refiner.0", False, 1, 32, 0, 0, seed=4)

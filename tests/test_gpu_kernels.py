@@ -1,0 +1,130 @@
+"""GPU parity of the single steps, through the C ABI, against the CPU oracle.
+
+Tolerances: integer outputs (positions, packed weights) bit-exact; fp32
+elementwise steps to fp32 rounding; bf16-output GEMM to bf16 rounding of the
+output (rel-L2 <= 4e-3, i.e. ~2^-8); attention rel-L2 <= 1e-2 (P is rounded to
+bf16 before the PV product, ~2^-9 per weight)."""
+import numpy as np
+import pytest
+
+from gpu_util import assert_parity, bits_f64, dev_bits, host_f64, rel_l2, require_gpu, torch
+import zimage_inputs as zi
+from oracle import scheduler_ref as sch, zimage_ref as ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+    from stream_diffusion_transformer_b200 import abi
+    abi.lib()
+    abi.clear_device_status()
+    yield
+    assert abi.device_status() == 0
+
+
+@pytest.fixture(scope="module")
+def M():
+    from stream_diffusion_transformer_b200 import abi, model
+    return abi, model
+
+
+@pytest.mark.parametrize("s_txt,gh,gw", [(32, 64, 64), (128, 32, 32), (512, 128, 128), (1, 1, 1), (7, 3, 5)])
+def test_positions_bit_exact(M, s_txt, gh, gw):
+    abi, model = M
+    got = model.positions(s_txt, gh, gw).cpu().numpy()
+    np.testing.assert_array_equal(got, ref.position_ids(s_txt, gh, gw))
+
+
+def test_rope_table(M):
+    abi, model = M
+    cfg = abi.config_default()
+    pos = model.positions(32, 64, 64)
+    tab = model.rope_table(cfg, pos).cpu().numpy().astype(np.float64)
+    ang = ref.rope_angles(ref.position_ids(32, 64, 64))
+    np.testing.assert_allclose(tab[..., 0], np.cos(ang), rtol=0, atol=2e-7)
+    np.testing.assert_allclose(tab[..., 1], np.sin(ang), rtol=0, atol=2e-7)
+
+
+@pytest.mark.parametrize("cfg_guidance", [None, 4.0])
+def test_euler_step(M, cfg_guidance):
+    abi, model = M
+    rng = np.random.default_rng(0)
+    n = 16 * 128 * 128 + 3  # ragged tail
+    x = rng.standard_normal(n).astype(np.float32)
+    yc = rng.standard_normal(n).astype(np.float32)
+    yu = rng.standard_normal(n).astype(np.float32)
+    sig = sch.sigmas(8)
+    xt = torch.from_numpy(x).cuda()
+    model.euler_step(xt, torch.from_numpy(yc).cuda(), None if cfg_guidance is None else torch.from_numpy(yu).cuda(),
+                     cfg_guidance or 0.0, sig[2], sig[3])
+    y = yc.astype(np.float64) if cfg_guidance is None else sch.cfg_combine(yc.astype(np.float64), yu, cfg_guidance)
+    want = sch.euler_step(x.astype(np.float64), y, sig[2], sig[3])
+    np.testing.assert_allclose(xt.cpu().numpy(), want, rtol=2e-6, atol=2e-6)
+
+
+def test_pack_qkv_and_ffn_bit_exact(M):
+    abi, model = M
+    D, F = 256, 688
+    wq, wk, wv = (zi.make_matrix((D, D), 1, i) for i in range(3))
+    got = model.pack_qkv(dev_bits(wq), dev_bits(wk), dev_bits(wv)).view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, np.concatenate([wq, wk, wv]))
+    w1, w3 = zi.make_matrix((F, D), 2, 0), zi.make_matrix((F, D), 2, 1)
+    w2 = zi.make_matrix((D, F), 2, 2)
+    Fp = abi.ffn_padded(F)
+    w13 = torch.empty((2 * Fp, D), dtype=torch.bfloat16, device="cuda")
+    w2p = torch.empty((D, Fp), dtype=torch.bfloat16, device="cuda")
+    abi.call("zi_pack_ffn", model._p(dev_bits(w1)), model._p(dev_bits(w3)), model._p(dev_bits(w2)), F, D,
+             model._p(w13), model._p(w2p), model._stream())
+    torch.cuda.synchronize()
+    g13 = w13.view(torch.int16).cpu().numpy().view(np.uint16)
+    g2 = w2p.view(torch.int16).cpu().numpy().view(np.uint16)
+    pad = lambda a: np.concatenate([a, np.zeros((Fp - F, D), np.uint16)])
+    want13 = np.stack([pad(w1).reshape(Fp // 128, 128, D), pad(w3).reshape(Fp // 128, 128, D)], 1).reshape(2 * Fp, D)
+    np.testing.assert_array_equal(g13, want13)
+    np.testing.assert_array_equal(g2, np.concatenate([w2, np.zeros((D, Fp - F), np.uint16)], 1))
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 64), (96, 768, 256), (127, 256, 128), (129, 512, 192),
+                                   (300, 1536, 256), (1152, 3840, 3840), (4128, 1280, 640)])
+def test_gemm_bf16(M, m, n, k):
+    abi, model = M
+    a = zi.make_matrix((m, k), 3, 0)
+    b = zi.make_matrix((n, k), 3, 1, std=0.05)
+    c = model.gemm(dev_bits(a), dev_bits(b))
+    torch.cuda.synchronize()
+    want = bits_f64(a) @ bits_f64(b).T
+    got = host_f64(c)
+    assert rel_l2(got, want) <= 4e-3
+    assert np.abs(got - want).max() <= 1e-2 * np.abs(want).max() + 1e-6
+
+
+@pytest.mark.parametrize("batch,seq,heads", [(1, 96, 2), (1, 128, 1), (2, 200, 2), (1, 1152, 4), (1, 33, 3)])
+def test_attention(M, batch, seq, heads):
+    abi, model = M
+    D = heads * 128
+    qkv = zi.make_matrix((batch * seq, 3 * D), 4, seq)
+    out = model.attention(dev_bits(qkv), batch, seq, heads)
+    torch.cuda.synchronize()
+    got = host_f64(out).reshape(batch, seq, heads, 128)
+    x = bits_f64(qkv).reshape(batch, seq, 3, heads, 128)
+    for b in range(batch):
+        want = ref.attention(x[b, :, 0], x[b, :, 1], x[b, :, 2])
+        assert_parity(got[b], want, rel=1e-2, cos=0.9999, what=f"attention b={b}")
+
+
+def test_attention_sharp_scores(M):
+    """Large logits: the running max moves by far more than 2^8 between key tiles."""
+    abi, model = M
+    seq, heads = 512, 1
+    D = 128
+    qkv = zi.bf16_bits_to_f32(zi.make_matrix((seq, 3 * D), 5, 0)).reshape(seq, 3, D)
+    qkv[:, 0] *= 4.0
+    qkv[:, 1] *= np.linspace(0.5, 6.0, seq, dtype=np.float32)[:, None]  # later keys dominate
+    bits = zi.f32_to_bf16_bits(qkv.reshape(seq, 3 * D))
+    out = model.attention(dev_bits(bits), 1, seq, heads)
+    torch.cuda.synchronize()
+    x = bits_f64(bits).reshape(seq, 3, 1, 128)
+    want = ref.attention(x[:, 0], x[:, 1], x[:, 2])
+    assert_parity(host_f64(out).reshape(seq, 1, 128), want, rel=1e-2, cos=0.9999, what="sharp attention")

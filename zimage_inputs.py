@@ -202,3 +202,14 @@ def make_cond(d: Dims, batch: int, seed: int = 0, std: float = 0.07) -> np.ndarr
     """A conditioning vector c N(0, std^2), fp32 [B, ada_dim], for single-block workloads."""
     return (_rng(seed, LATENT_STREAM, 2).standard_normal(size=(batch, d.ada_dim), dtype=np.float32)
             * np.float32(std))
+
+
+MATRIX_STREAM = 4
+
+
+def make_matrix(shape: Sequence[int], seed: int = 0, index: int = 0, std: float = 1.0) -> np.ndarray:
+    """A generic N(0, std^2) tensor rounded to bf16 (bits), for single-kernel checks."""
+    v = _rng(seed, MATRIX_STREAM, index).standard_normal(size=tuple(shape), dtype=np.float32)
+    if std != 1.0:
+        v *= np.float32(std)
+    return f32_to_bf16_bits(v)
