@@ -68,15 +68,17 @@ def test_pack_qkv_and_ffn_bit_exact(M):
     abi, model = M
     D, F = 256, 688
     wq, wk, wv = (zi.make_matrix((D, D), 1, i) for i in range(3))
-    got = model.pack_qkv(dev_bits(wq), dev_bits(wk), dev_bits(wv)).view(torch.int16).cpu().numpy().view(np.uint16)
+    dq, dk, dv = dev_bits(wq), dev_bits(wk), dev_bits(wv)
+    got = model.pack_qkv(dq, dk, dv).view(torch.int16).cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(got, np.concatenate([wq, wk, wv]))
     w1, w3 = zi.make_matrix((F, D), 2, 0), zi.make_matrix((F, D), 2, 1)
     w2 = zi.make_matrix((D, F), 2, 2)
     Fp = abi.ffn_padded(F)
     w13 = torch.empty((2 * Fp, D), dtype=torch.bfloat16, device="cuda")
     w2p = torch.empty((D, Fp), dtype=torch.bfloat16, device="cuda")
-    abi.call("zi_pack_ffn", model._p(dev_bits(w1)), model._p(dev_bits(w3)), model._p(dev_bits(w2)), F, D,
-             model._p(w13), model._p(w2p), model._stream())
+    d1, d3, d2 = dev_bits(w1), dev_bits(w3), dev_bits(w2)  # kept alive until the copies ran
+    abi.call("zi_pack_ffn", model._p(d1), model._p(d3), model._p(d2), F, D, model._p(w13), model._p(w2p),
+             model._stream())
     torch.cuda.synchronize()
     g13 = w13.view(torch.int16).cpu().numpy().view(np.uint16)
     g2 = w2p.view(torch.int16).cpu().numpy().view(np.uint16)
