@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark: Z-Image S3-DiT full transformer forward at 4,128 tokens on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one full forward (2 noise-refiner + 2 context-refiner + 30 main
+blocks, embedders and final layer) of a 1024x1024 image (latent 16x128x128 ->
+4,096 image tokens) with 32 text tokens, batch 1, on random-init bf16 weights
+(6,154,908,736 parameters, seeded) resident in HBM.  The value is algorithmic
+TFLOP/s (per block 8SD^2 + 6SDF + 4S^2D, plus embedders and final layer).
+
+--gpus N > 1 runs N independent replicas (one process per GPU, launched by
+torch.distributed.run); the forward has no exchange step, so there is no
+data-path collective: barriers and the max-over-ranks timing use NCCL.
+
+--impl reference times the CPU oracle (NumPy, fp64) on the host cores, each
+step one main block of the same 4,128-token workload (a bounded sample).
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import zimage_inputs as zi  # noqa: E402
+
+METRIC = "DiT forward ms & TFLOP/s at 4,128 tokens; % of B200 bf16 tensor peak"
+WORKLOAD = ("full stack one forward: 2 context-refiner + 2 noise-refiner + 30 main blocks, "
+            "1024x1024 -> 4,096 image + 32 text = 4,128 tokens, batch 1")
+LAT_H = LAT_W = 128
+S_TXT = 32
+T_VALUE = 0.5
+SEED = 0
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def block_flops(S: int, D: int, F: int) -> float:
+    return 8.0 * S * D * D + 6.0 * S * D * F + 4.0 * S * S * D
+
+
+def forward_flops(d: zi.Dims, s_img: int, s_txt: int, batch: int = 1) -> float:
+    D, F = d.dim, d.ffn
+    S = s_img + s_txt
+    f = d.n_noise * block_flops(s_img, D, F) + d.n_ctx * block_flops(s_txt, D, F) + d.n_main * block_flops(S, D, F)
+    f += 2.0 * s_img * d.patch_dim * D + 2.0 * s_txt * d.cap_dim * D + 2.0 * s_img * D * d.patch_dim
+    return batch * f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "stream_diffusion_transformer_b200", "csrc")
+    for name in sorted(os.listdir(cdir)):
+        with open(os.path.join(cdir, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        rec = json.load(fh)
+    e = rec.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        mx = float(rows[0][2])
+        load = [float(r[1]) for r in rows if float(r[3]) > 250.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample():
+    """The CPU oracle's bounded sample: one main block of the 4,128-token workload (fp64)."""
+    from oracle import zimage_ref as ref
+    d = zi.FULL
+    s_img = (LAT_H // 2) * (LAT_W // 2)
+    S = s_img + S_TXT
+    bits = zi.make_weights(d, seed=SEED, keys=[k for k, _, _ in zi.block_specs("layers.0", d, True)], threads=8)
+    W = ref.Weights(bits)
+    x = zi.make_stream(d, 1, S, seed=SEED)[0].astype(np.float64)
+    c = zi.make_cond(d, 1, seed=SEED)[0].astype(np.float64)
+    ang = ref.rope_angles(ref.position_ids(S_TXT, LAT_H // 2, LAT_W // 2), d.rope_axes)
+
+    def step():
+        return ref.block_forward(x, W, "layers.0", d, ang, c)
+
+    return step, block_flops(S, d.dim, d.ffn), f"one main block (full width, {S} tokens, fp64 NumPy)"
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    step, flops, sample = oracle_sample()
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": (LAT_H // 2) * (LAT_W // 2) + S_TXT, "batch": 1,
+                   "sample_per_step": sample, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from stream_diffusion_transformer_b200 import abi, model
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    d = zi.FULL
+    cfg = model.make_config(d)
+    s_img = (LAT_H // 2) * (LAT_W // 2)
+    S = s_img + S_TXT
+    flops = forward_flops(d, s_img, S_TXT)
+    abi.clear_device_status()
+
+    # weights: generated on rank 0's host threads, broadcast to the other ranks
+    threads = max(1, min(32, (os.cpu_count() or 8)))
+
+    def fetch(keys):
+        if world == 1 or rank == 0:
+            out = zi.make_weights(d, seed=SEED, keys=keys, threads=threads)
+        else:
+            out = {}
+        if world > 1:
+            specs = {k: s for k, s, _ in zi.weight_specs(d)}
+            res = {}
+            for k in keys:
+                t = (torch.from_numpy(out[k].view(np.int16)).to(dev) if rank == 0
+                     else torch.empty(specs[k], dtype=torch.int16, device=dev))
+                dist.broadcast(t, 0)
+                res[k] = t.cpu().numpy().view(np.uint16)
+            return res
+        return out
+
+    t_load = time.perf_counter()
+    dit = model.DiT(cfg, fetch, device=dev)
+    load_s = time.perf_counter() - t_load
+
+    lat = torch.from_numpy(zi.make_latent(d, 1, LAT_H, LAT_W, seed=SEED)).to(dev)
+    txt = torch.from_numpy(zi.make_text(d, 1, S_TXT, seed=SEED).view(np.int16)).to(dev).view(torch.bfloat16)
+    tt = torch.full((1,), T_VALUE, dtype=torch.float32, device=dev)
+    out = torch.empty_like(lat)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        dit.forward(lat, tt, txt, out)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K forwards, inputs resident in HBM
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        with abi.Profile(capacity=600 * args.steps + 64) as prof:
+            start.record(stream)
+            for _ in range(args.steps):
+                dit.forward(lat, tt, txt, out)
+            end.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = abi.device_status()
+    if status != 0:
+        raise RuntimeError(f"device pipeline timeout (code {status}) during the timed region")
+    out_finite = bool(torch.isfinite(out).all().item())
+
+    # ---- end to end through the public API: pinned host inputs in, result out, every step
+    h_lat = torch.from_numpy(zi.make_latent(d, 1, LAT_H, LAT_W, seed=SEED)).pin_memory()
+    h_txt = torch.from_numpy(zi.make_text(d, 1, S_TXT, seed=SEED).view(np.int16)).pin_memory()
+    h_t = torch.full((1,), T_VALUE, dtype=torch.float32).pin_memory()
+    h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    d_lat, d_txt, d_t = torch.empty_like(lat), torch.empty(txt.shape, dtype=torch.int16, device=dev), torch.empty_like(tt)
+
+    def e2e_step():
+        d_lat.copy_(h_lat, non_blocking=True)
+        d_txt.copy_(h_txt, non_blocking=True)
+        d_t.copy_(h_t, non_blocking=True)
+        dit.forward(d_lat, d_t, d_txt.view(torch.bfloat16), out)
+        h_out.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    h2d = h_lat.numel() * 4 + h_txt.numel() * 2 + h_t.numel() * 4
+    d2h = h_out.numel() * 4
+
+    if rank != 0:
+        return
+
+    # ---- per-kernel durations from the events recorded between launches in the timed region
+    per_step = len(prof.kinds) // args.steps
+    table = {}
+    for k, m in zip(prof.kinds, prof.ms):
+        e = table.setdefault(k, {"launches": 0, "ms": 0.0})
+        e["launches"] += 1
+        e["ms"] += m
+    total_ms = sum(prof.ms)
+    for k in table:
+        table[k]["share"] = table[k]["ms"] / total_ms
+        table[k]["ms_per_launch"] = table[k]["ms"] / table[k]["launches"]
+
+    def main_block_launches(kind):
+        """Durations of `kind` in the 30 main blocks (4,128 rows), per forward in launch order."""
+        out_ms = []
+        for sidx in range(args.steps):
+            seq = [(k, m) for k, m in zip(prof.kinds[sidx * per_step:(sidx + 1) * per_step],
+                                          prof.ms[sidx * per_step:(sidx + 1) * per_step]) if k == kind]
+            out_ms += [m for _, m in seq[-d.n_main:]]
+        return out_ms
+
+    peaks, peak_src = load_peaks()
+    peak_tensor = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    ffn_ms = statistics.mean(main_block_launches("gemm_ffn_up_swiglu"))
+    ffn_flops = 2.0 * S * d.dim * (2 * d.ffn)
+    ffn_tflops = ffn_flops / (ffn_ms * 1e-3) / 1e12
+    att_ms = statistics.mean(main_block_launches("attention"))
+    att_tflops = 4.0 * S * S * d.dim / (att_ms * 1e-3) / 1e12
+    per_kernel_roof = {}
+    for kind, fl in (("gemm_qkv_qknorm_rope", 6.0 * S * d.dim ** 2), ("attention", 4.0 * S * S * d.dim),
+                     ("gemm_out_proj", 2.0 * S * d.dim ** 2), ("gemm_ffn_up_swiglu", ffn_flops),
+                     ("gemm_ffn_down", 2.0 * S * d.dim * d.ffn)):
+        m = statistics.mean(main_block_launches(kind))
+        per_kernel_roof[kind] = {"ms_per_launch": m, "tflops": fl / (m * 1e-3) / 1e12,
+                                 "frac": fl / (m * 1e-3) / 1e12 / peak_tensor}
+    for kind, bytes_per_row in (("post_norm_residual", 4 * d.dim * 2 + 2 * d.dim * 2),):
+        m = statistics.mean(main_block_launches(kind))
+        gbs = bytes_per_row * S / (m * 1e-3) / 1e9
+        per_kernel_roof[kind] = {"ms_per_launch": m, "gbs": gbs, "frac": gbs / float(peaks["hbm_gbs"])}
+
+    clk = clocks.summary()
+    value = flops * world * args.steps / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD, "tokens": S, "batch": 1, "image": "1024x1024", "text_tokens": S_TXT,
+            "t": T_VALUE, "params": sum(int(np.prod(s)) for _, s, _ in zi.weight_specs(d)),
+            "flops_per_step": flops, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "no flush: every step streams all 12.3 GB of weights (> 126 MB L2) from HBM",
+            "cuda_graph": False, "weight_load_s": round(load_s, 1),
+        },
+        "tensor_peak_frac": value / world / peak_tensor,
+        "roofline": {
+            "kernel": "gemm_ffn_up_swiglu (main block, M=4128, N=20480, K=3840)",
+            "bound": "tensor", "achieved": ffn_tflops, "peak": peak_tensor, "unit": "TFLOP/s",
+            "frac": ffn_tflops / peak_tensor,
+            "traffic": recorded_traffic("gemm_ffn_up_swiglu"),
+            "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+            "algorithmic_flops_per_launch": ffn_flops,
+        },
+        "attention_roofline": {"achieved": att_tflops, "peak": peak_tensor, "frac": att_tflops / peak_tensor,
+                               "unit": "TFLOP/s", "ms_per_launch": att_ms},
+        "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in e.items()}
+                    for k, e in sorted(table.items(), key=lambda kv: -kv[1]["ms"])},
+        "kernel_rooflines": per_kernel_roof,
+        "gpu_launches": len(prof.kinds),
+        "e2e": {"value": flops * world * args.steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps},
+        "clocks": clk,
+        "output_finite": out_finite,
+        "published_context": {"ms": 22500.0, "hardware": "Apple M1 Pro", "precision": "int8 ConvRot",
+                              "source": "Z-Image-Turbo repackaged for H3ddle, Measured performance"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        step, sflops, sample = oracle_sample()
+        t0 = time.perf_counter()
+        step()
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": sflops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -227,6 +227,41 @@ ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c,
  * d_out bf16 [batch*seq, heads*128]. */
 ZI_API int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads, zi_stream_t stream);
 
+/* ---------------------------------------------------------------- launch profiling */
+
+/* Kernel identities reported by zi_profile_end. */
+enum zi_kernel_kind {
+  ZI_KERNEL_GEMM_QKV = 1,       /* QKV projection + QK-RMSNorm + RoPE epilogue */
+  ZI_KERNEL_ATTENTION = 2,      /* flash attention */
+  ZI_KERNEL_GEMM_OUT = 3,       /* attention output projection */
+  ZI_KERNEL_GEMM_FFN_UP = 4,    /* w1|w3 projection + SwiGLU epilogue */
+  ZI_KERNEL_GEMM_FFN_DOWN = 5,  /* w2 projection */
+  ZI_KERNEL_POST_NORM = 6,      /* post-norm + gated residual + next pre-norm */
+  ZI_KERNEL_PRE_NORM = 7,       /* RMSNorm x (1 + scale) -> bf16 */
+  ZI_KERNEL_ADALN = 8,          /* all adaLN projections */
+  ZI_KERNEL_TIMESTEP = 9,       /* timestep sinusoid + MLP */
+  ZI_KERNEL_ROPE = 10,          /* RoPE cos/sin table */
+  ZI_KERNEL_POSITIONS = 11,     /* position ids */
+  ZI_KERNEL_PATCHIFY = 12,      /* latent -> patch tokens */
+  ZI_KERNEL_GEMM_EMBED = 13,    /* x_embedder / cap_embedder projection */
+  ZI_KERNEL_GEMM_FINAL = 14,    /* final linear + unpatchify */
+  ZI_KERNEL_EULER = 15,         /* Euler / CFG step */
+  ZI_KERNEL_GEMM = 16           /* zi_gemm_bf16 */
+};
+
+/* Start recording launch timings on this host thread: from the next kernel the
+ * library enqueues, a timing event is recorded before the first kernel and after
+ * every kernel (up to `capacity` kernels), on the launching stream.  Creates
+ * capacity + 1 CUDA events (no device memory).  ZI_ERR_ARG if already started. */
+ZI_API int zi_profile_begin(int capacity);
+
+/* Stop recording: waits for the last recorded event, writes per-launch times in
+ * milliseconds (time from the previous marker to this kernel's end marker) to
+ * h_ms and zi_kernel_kind ids to h_kinds (up to `capacity` entries each; either
+ * may be NULL), the number of launches to *h_count (-1 if more kernels ran than
+ * the capacity given to zi_profile_begin), and destroys the events. */
+ZI_API int zi_profile_end(float* h_ms, int* h_kinds, int capacity, int* h_count);
+
 /* ---------------------------------------------------------------- device status */
 
 /* Reads (synchronously) the device error word of the current device: ZI_OK, or

@@ -210,6 +210,38 @@ def block_forward(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: np.nd
     return x2
 
 
+def block_forward_rows(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: np.ndarray,
+                       c: Optional[np.ndarray], rows: np.ndarray) -> np.ndarray:
+    """block_forward(x, ...)[rows], computed for those query rows only.
+
+    Keys and values come from every row of x (the attention is over the whole
+    sequence); every other step is per row, so only the selected rows go
+    through the query projection, attention, output projection and FFN.
+    """
+    S, D = x.shape
+    H, hd = d.heads, d.head_dim
+    if c is not None:
+        scale_msa, gate_msa, scale_mlp, gate_mlp = adaln(c, W, prefix)
+    else:
+        scale_msa = scale_mlp = 0.0
+        gate_msa = gate_mlp = 1.0
+    a = f"{prefix}.attention"
+    h = rms_norm(x, W(f"{prefix}.attention_norm1.weight")) * (1.0 + scale_msa)
+    k = apply_rope(rms_norm(linear(h, W(f"{a}.to_k.weight")).reshape(S, H, hd), W(f"{a}.norm_k.weight")), angles)
+    v = linear(h, W(f"{a}.to_v.weight")).reshape(S, H, hd)
+    hr = h[rows]
+    q = linear(hr, W(f"{a}.to_q.weight")).reshape(len(rows), H, hd)
+    q = apply_rope(rms_norm(q, W(f"{a}.norm_q.weight")), angles[rows])
+    att = attention(q, k, v).reshape(len(rows), D)
+    o = linear(att, W(f"{a}.to_out.weight"))
+    x1 = x[rows] + gate_msa * rms_norm(o, W(f"{prefix}.attention_norm2.weight"))
+    h2 = rms_norm(x1, W(f"{prefix}.ffn_norm1.weight")) * (1.0 + scale_mlp)
+    ff = f"{prefix}.feed_forward"
+    u = silu(linear(h2, W(f"{ff}.w1.weight"))) * linear(h2, W(f"{ff}.w3.weight"))
+    f = linear(u, W(f"{ff}.w2.weight"))
+    return x1 + gate_mlp * rms_norm(f, W(f"{prefix}.ffn_norm2.weight"))
+
+
 def final_layer(x_img: np.ndarray, W: Weights, c: np.ndarray) -> np.ndarray:
     """LayerNorm(x) * (1 + Linear(SiLU(c))) -> Linear to p*p*C features."""
     s = linear(silu(c), W("final_layer.adaLN_modulation.weight"), W("final_layer.adaLN_modulation.bias"))

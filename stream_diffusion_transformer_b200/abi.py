@@ -67,6 +67,8 @@ _SIGS = {
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
     "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_profile_begin": (c_int, [c_int]),
+    "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),
     "zi_device_status": (c_int, [POINTER(c_int)]),
     "zi_clear_device_status": (c_int, []),
 }
@@ -142,6 +144,46 @@ def device_status() -> int:
 
 def clear_device_status() -> None:
     call("zi_clear_device_status")
+
+
+KERNEL_NAMES = {
+    1: "gemm_qkv_qknorm_rope", 2: "attention", 3: "gemm_out_proj", 4: "gemm_ffn_up_swiglu",
+    5: "gemm_ffn_down", 6: "post_norm_residual", 7: "pre_norm", 8: "adaln_gemv", 9: "timestep_mlp",
+    10: "rope_table", 11: "positions", 12: "patchify", 13: "gemm_embed", 14: "gemm_final_unpatchify",
+    15: "euler", 16: "gemm",
+}
+
+
+class Profile:
+    """Context manager recording the duration of every library kernel launched inside it."""
+
+    def __init__(self, capacity: int = 4096):
+        self.capacity = capacity
+        self.ms = []
+        self.kinds = []
+
+    def __enter__(self):
+        call("zi_profile_begin", self.capacity)
+        return self
+
+    def __exit__(self, *exc):
+        ms = (c_float * self.capacity)()
+        kinds = (c_int * self.capacity)()
+        n = c_int(0)
+        call("zi_profile_end", ms, kinds, self.capacity, ctypes.byref(n))
+        if n.value < 0:
+            raise RuntimeError("profile capacity exceeded")
+        self.ms = list(ms[:n.value])
+        self.kinds = [KERNEL_NAMES.get(k, str(k)) for k in kinds[:n.value]]
+        return False
+
+    def by_kernel(self):
+        out = {}
+        for k, m in zip(self.kinds, self.ms):
+            e = out.setdefault(k, [0, 0.0])
+            e[0] += 1
+            e[1] += m
+        return out
 
 
 def exported_symbols():

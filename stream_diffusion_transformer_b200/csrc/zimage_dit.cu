@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "zi_attention.cuh"
 #include "zi_common.cuh"
@@ -102,7 +103,38 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline int launch_status() { return cudaGetLastError() == cudaSuccess ? ZI_OK : ZI_ERR_CUDA; }
+// ---------------------------------------------------------------- launch profiling
+// While enabled (zi_profile_begin .. zi_profile_end, per host thread) an event
+// is recorded on the launching stream before the first kernel and after every
+// kernel, so consecutive events bracket each launch.
+struct Prof {
+  bool on = false, started = false, overflow = false;
+  int cap = 0, n = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> kind;
+};
+thread_local Prof g_prof;
+
+inline void prof_pre(cudaStream_t st) {
+  if (g_prof.on && !g_prof.started) {
+    cudaEventRecord(g_prof.ev[0], st);
+    g_prof.started = true;
+  }
+}
+
+// Status of the launch just made (+ the profiling marker after it).
+inline int launched(int kind, cudaStream_t st) {
+  if (cudaGetLastError() != cudaSuccess) return ZI_ERR_CUDA;
+  if (g_prof.on) {
+    if (g_prof.n < g_prof.cap) {
+      cudaEventRecord(g_prof.ev[g_prof.n + 1], st);
+      g_prof.kind[g_prof.n++] = kind;
+    } else {
+      g_prof.overflow = true;
+    }
+  }
+  return ZI_OK;
+}
 
 #define ZI_TRY(expr)          \
   do {                        \
@@ -125,7 +157,7 @@ enum KernelBit : unsigned {
 constexpr int kStages = 4;
 
 template <int BN, int EPI>
-int run_gemm(DevInfo* dev, unsigned bit, const uint16_t* A, const uint16_t* B, int M, int N, int K,
+int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint16_t* B, int M, int N, int K,
              const EpiParams& ep, cudaStream_t st) {
   using L = GemmSmem<BN, kStages>;
   if (M <= 0) return ZI_OK;
@@ -137,8 +169,9 @@ int run_gemm(DevInfo* dev, unsigned bit, const uint16_t* A, const uint16_t* B, i
   ZI_TRY(ensure_smem(dev, bit, kern, int(L::kBytes)));
   const int tiles = ((M + 127) / 128) * (N / BN);
   const int grid = tiles < dev->sms ? tiles : dev->sms;
+  prof_pre(st);
   kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, N, K, ep);
-  return launch_status();
+  return launched(kind, st);
 }
 
 EpiParams epi_plain(void* out, int ldo) {
@@ -171,8 +204,9 @@ int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out
   }
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(128.0));
   dim3 grid(qt, heads, batch);
+  prof_pre(st);
   attention_kernel<<<grid, 192, attn::kSmemBytes, st>>>(tm, p);
-  return launch_status();
+  return launched(ZI_KERNEL_ATTENTION, st);
 }
 
 // ---------------------------------------------------------------- row kernels
@@ -181,14 +215,16 @@ template <typename TIn>
 int run_rms_mod(const TIn* x, int rows, int D, const uint16_t* gain, const float* scale, int scale_ld, RowMap map,
                 int row_off, float eps, uint16_t* h, cudaStream_t st) {
   if (rows <= 0) return ZI_OK;
+  prof_pre(st);
   rms_mod_kernel<TIn><<<rows, kRowThreads, 0, st>>>(x, D, gain, scale, scale_ld, map, row_off, eps, h);
-  return launch_status();
+  return launched(ZI_KERNEL_PRE_NORM, st);
 }
 
 int run_post(const PostParams& p, int rows, cudaStream_t st) {
   if (rows <= 0) return ZI_OK;
+  prof_pre(st);
   post_residual_kernel<<<rows, kRowThreads, 0, st>>>(p);
-  return launch_status();
+  return launched(ZI_KERNEL_POST_NORM, st);
 }
 
 // ---------------------------------------------------------------- workspace
@@ -299,9 +335,9 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   eq.dim = D;
   eq.row_off = b.row_off;
   eq.map = b.map;
-  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st)));
+  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st)));
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len, st));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, b.att, b.w->w_out, b.rows, D, D, epi_plain(b.o, D), st)));
+  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D, epi_plain(b.o, D), st)));
   PostParams pa;
   memset(&pa, 0, sizeof(pa));
   pa.x_in = b.x_in;
@@ -322,9 +358,9 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   pa.eps = eps;
   pa.eps_ln = b.cfg->final_eps;
   ZI_TRY(run_post(pa, b.rows, st));
-  ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, b.h, b.w->w13, b.rows, 2 * Fp, D, epi_plain(b.u, Fp),
+  ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp, D, epi_plain(b.u, Fp),
                                     st)));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, b.u, b.w->w2, b.rows, D, Fp, epi_plain(b.o, D), st)));
+  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp, epi_plain(b.o, D), st)));
   PostParams pf = pa;
   pf.x_in = b.x_out;
   pf.g_post = b.w->g_ffn2;
@@ -341,16 +377,18 @@ int run_ada(const AdaSegs& segs, const float* c, const float* silu_c, int batch,
   int max_rows = 0;
   for (int i = 0; i < segs.n; ++i) max_rows = segs.rows[i] > max_rows ? segs.rows[i] : max_rows;
   dim3 grid((max_rows + 63) / 64, segs.n);
+  prof_pre(st);
   ada_gemv_kernel<<<grid, 256, 0, st>>>(segs, c, silu_c, batch, out_ld, out);
-  return launch_status();
+  return launched(ZI_KERNEL_ADALN, st);
 }
 
 int run_rope(const zi_config& cfg, const int32_t* pos, int n, float2* out, cudaStream_t st) {
   const int pairs = cfg.head_dim / 2;
   const int total = n * pairs;
+  prof_pre(st);
   rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(pos, n, cfg.rope_axes[0], cfg.rope_axes[1],
                                                            cfg.rope_axes[2], double(cfg.rope_theta), out);
-  return launch_status();
+  return launched(ZI_KERNEL_ROPE, st);
 }
 
 }  // namespace
@@ -471,9 +509,10 @@ int zi_positions(int s_txt, int grid_h, int grid_w, int32_t* d_pos, zi_stream_t 
   ZI_TRY(current_device(&dev));
   const int n = grid_h * grid_w + s_txt;
   if (n == 0) return ZI_OK;
-  positions_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(s_txt, grid_h, grid_w,
-                                                                                         d_pos);
-  return launch_status();
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  prof_pre(st);
+  positions_kernel<<<(n + 255) / 256, 256, 0, st>>>(s_txt, grid_h, grid_w, d_pos);
+  return launched(ZI_KERNEL_POSITIONS, st);
 }
 
 int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, float* d_cos_sin, zi_stream_t stream) {
@@ -491,7 +530,7 @@ int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m,
   if (k % 64 || n % 256) return ZI_ERR_SHAPE;
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
-  return run_gemm<256, EPI_BF16>(dev, BIT_GEMM_BF16, d_a, d_b, m, n, k, epi_plain(d_c, n),
+  return run_gemm<256, EPI_BF16>(dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM, d_a, d_b, m, n, k, epi_plain(d_c, n),
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -627,9 +666,10 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
   {
     const int smem = (cfg->t_freq + cfg->t_mid) * 4;
     if (smem > 48 * 1024) return ZI_ERR_SHAPE;
+    prof_pre(st);
     timestep_mlp_kernel<<<batch, 256, smem, st>>>(d_t, cfg->t_scale, cfg->t_freq, cfg->t_mid, 256, w->t_w1,
                                                   w->t_b1, w->t_w2, w->t_b2, c, silu_c);
-    ZI_TRY(launch_status());
+    ZI_TRY(launched(ZI_KERNEL_TIMESTEP, st));
     AdaSegs segs;
     memset(&segs, 0, sizeof(segs));
     int k = 0;
@@ -658,23 +698,25 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
   const float* final_scale = mod + size_t(n_mod) * 4 * D;
 
   // positions and RoPE table of one sequence [image; text]
+  prof_pre(st);
   positions_kernel<<<(S + 255) / 256, 256, 0, st>>>(s_txt, gh, gw, pos);
-  ZI_TRY(launch_status());
+  ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
   ZI_TRY(run_rope(*cfg, pos, S, rope, st));
 
   // embedders: image rows [0, rows_img), text rows [rows_img, rows)
   {
     const size_t n = size_t(rows_img) * 64;
+    prof_pre(st);
     patchify_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(d_latent, batch, cfg->in_ch, lat_h, lat_w, tok);
-    ZI_TRY(launch_status());
+    ZI_TRY(launched(ZI_KERNEL_PATCHIFY, st));
     EpiParams ex = epi_plain(x, D);
     ex.bias = w->x_emb_b;
-    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, tok, w->x_emb_w, rows_img, D, 64, ex, st)));
+    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, tok, w->x_emb_w, rows_img, D, 64, ex, st)));
     ZI_TRY(run_rms_mod<uint16_t>(d_txt, rows_txt, cfg->cap_dim, w->cap_norm, nullptr, 0, map, rows_img, eps, capn,
                                  st));
     EpiParams ec = epi_plain(x + size_t(rows_img) * D, D);
     ec.bias = w->cap_b;
-    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, capn, w->cap_w, rows_txt, D, cfg->cap_dim, ec, st)));
+    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, capn, w->cap_w, rows_txt, D, cfg->cap_dim, ec, st)));
   }
 
   BlockCtx base;
@@ -767,7 +809,7 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
     ef.lat_c = cfg->in_ch;
     ef.lat_h = lat_h;
     ef.lat_w = lat_w;
-    ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, h, w->final_w, rows_img, 4 * cfg->in_ch, D, ef, st)));
+    ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, ZI_KERNEL_GEMM_FINAL, h, w->final_w, rows_img, 4 * cfg->in_ch, D, ef, st)));
   }
   return ZI_OK;
 }
@@ -779,9 +821,10 @@ int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond
   ZI_TRY(current_device(&dev));
   if (n == 0) return ZI_OK;
   const float dt = float(sigma_next - sigma);
-  euler_kernel<<<unsigned((n + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      d_x, d_out_cond, d_out_uncond, guidance, dt, n);
-  return launch_status();
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  prof_pre(st);
+  euler_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(d_x, d_out_cond, d_out_uncond, guidance, dt, n);
+  return launched(ZI_KERNEL_EULER, st);
 }
 
 int zi_sigmas(int n_steps, double shift, double* h_sigmas) {
@@ -792,6 +835,42 @@ int zi_sigmas(int n_steps, double shift, double* h_sigmas) {
   }
   h_sigmas[n_steps] = 0.0;
   return ZI_OK;
+}
+
+int zi_profile_begin(int capacity) {
+  if (capacity <= 0) return ZI_ERR_ARG;
+  if (g_prof.on) return ZI_ERR_ARG;
+  Prof p;
+  p.ev.resize(size_t(capacity) + 1);
+  p.kind.assign(size_t(capacity), 0);
+  for (auto& e : p.ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (auto& f : p.ev)
+        if (f) cudaEventDestroy(f);
+      return ZI_ERR_CUDA;
+    }
+  }
+  p.cap = capacity;
+  p.on = true;
+  g_prof = std::move(p);
+  return ZI_OK;
+}
+
+int zi_profile_end(float* h_ms, int* h_kinds, int capacity, int* h_count) {
+  if (!g_prof.on) return ZI_ERR_ARG;
+  int st = ZI_OK;
+  const int n = g_prof.n;
+  if (h_count) *h_count = g_prof.overflow ? -1 : n;
+  if (n > 0 && cudaEventSynchronize(g_prof.ev[n]) != cudaSuccess) st = ZI_ERR_CUDA;
+  for (int i = 0; i < n && i < capacity && st == ZI_OK; ++i) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_prof.ev[i], g_prof.ev[i + 1]) != cudaSuccess) st = ZI_ERR_CUDA;
+    if (h_ms) h_ms[i] = ms;
+    if (h_kinds) h_kinds[i] = g_prof.kind[i];
+  }
+  for (auto& e : g_prof.ev) cudaEventDestroy(e);
+  g_prof = Prof();
+  return st;
 }
 
 int zi_device_status(int* h_code) {

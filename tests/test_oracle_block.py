@@ -95,6 +95,19 @@ def _block_setup(d=zi.TINY, seed=5, S=12):
     return bits, x, c, ang
 
 
+@pytest.mark.parametrize("modulated", [True, False])
+def test_block_rows_matches_block(modulated):
+    """The sampled-row form used at full size equals the whole block at those rows."""
+    d = zi.TINY
+    bits, x, c, ang = _block_setup(d, S=12)
+    W = ref.Weights(bits)
+    cc = c if modulated else None
+    rows = np.array([0, 5, 11, 7])
+    full = ref.block_forward(x, W, "layers.0", d, ang, cc)
+    np.testing.assert_allclose(ref.block_forward_rows(x, W, "layers.0", d, ang, cc, rows), full[rows],
+                               rtol=1e-12, atol=1e-14)
+
+
 def test_zero_modulation_gives_identity_block():
     """tanh(0) = 0 gates both residual updates off."""
     d = zi.TINY
