@@ -63,7 +63,8 @@ enum zi_status {
   ZI_ERR_WORKSPACE = -4, /* workspace missing or smaller than zi_*_workspace_size() */
   ZI_ERR_CUDA = -5,      /* a CUDA runtime/driver call failed (launch error etc.) */
   ZI_ERR_TIMEOUT = -6,   /* a kernel's bounded pipeline wait ran out (zi_device_status) */
-  ZI_ERR_DEVICE = -7     /* current device is not an sm_100 GPU */
+  ZI_ERR_DEVICE = -7,    /* current device is not an sm_100 GPU */
+  ZI_ERR_SCRATCH_LIMIT = -8 /* sizes need more than ZI_STATIC_SCRATCH_BYTES (zi_block_forward_noalloc) */
 };
 
 /* Sizes of one model variant.  zi_config_default() gives Z-Image's
@@ -204,6 +205,38 @@ ZI_API int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out
  * for s = linspace(1, 1/n_steps, n_steps), then 0 (z-image-turbo-mnn "Scheduler";
  * FastVideo handoff "Scheduler").  h_sigmas has n_steps + 1 entries. */
 ZI_API int zi_sigmas(int n_steps, double shift, double* h_sigmas);
+
+/* ---------------------------------------------------------------- fixed-scratch variant
+ * The pages describing the method have no counterpart to this entry point; it
+ * exists for callers that cannot allocate device memory.  Examples: a plugin
+ * running inside a host program whose memory manager owns all device memory
+ * and hands plugins no allocator, or a latency-critical loop that forbids
+ * cudaMalloc after start-up (cudaMalloc can synchronise the device and stall
+ * other work).  Such callers cannot provide the workspace zi_block_forward needs. */
+
+/* Bytes of the library's fixed device scratch (64 MiB).  Every GPU that loads the
+ * library holds this much device memory until the process exits. */
+#define ZI_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* zi_block_forward without a workspace argument: the scratch is a file-scope
+ * device array of ZI_STATIC_SCRATCH_BYTES inside the library.  The caller still
+ * passes (and owns) the inputs and the output; arguments mean what they mean
+ * for zi_block_forward.
+ *   - Allocates nothing: no cudaMalloc/cudaFree and no allocating library call.
+ *   - Sizes whose zi_block_workspace_size() exceeds ZI_STATIC_SCRATCH_BYTES are
+ *     rejected with ZI_ERR_SCRATCH_LIMIT before anything is enqueued (about 990
+ *     tokens of batch x seq at Z-Image's full width).
+ *   - The first call on each device looks up the scratch's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture on that device.
+ *   - Every call on a device shares the one scratch array, and it keeps the last
+ *     call's contents.  Nothing in it needs to start at zero (each call writes
+ *     every scratch byte it reads), but calls whose GPU work overlaps -- on
+ *     different streams, or from different host threads -- race on the scratch
+ *     and corrupt each other's results: serialise them. */
+ZI_API int zi_block_forward_noalloc(const zi_config* cfg, const zi_block_weights* w, const float* d_c,
+                                    const int32_t* d_pos, int batch, int seq, const float* d_x_in, float* d_x_out,
+                                    zi_stream_t stream);
 
 /* ---------------------------------------------------------------- single steps
  * The steps zi_block_forward / zi_model_forward chain, exposed for testing and

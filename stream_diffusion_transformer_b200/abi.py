@@ -14,6 +14,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzimage_d
 
 ZI_OK, ZI_ERR_ARG, ZI_ERR_SHAPE, ZI_ERR_ALIGN, ZI_ERR_WORKSPACE, ZI_ERR_CUDA, ZI_ERR_TIMEOUT, ZI_ERR_DEVICE = (
     0, -1, -2, -3, -4, -5, -6, -7)
+ZI_ERR_SCRATCH_LIMIT = -8
+STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class ZiError(RuntimeError):
@@ -59,6 +61,8 @@ _SIGS = {
     "zi_model_workspace_size": (c_int, [POINTER(ZiConfig), c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
     "zi_block_forward": (c_int, [POINTER(ZiConfig), POINTER(ZiBlockWeights), c_void_p, c_void_p, c_int, c_int,
                                  c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "zi_block_forward_noalloc": (c_int, [POINTER(ZiConfig), POINTER(ZiBlockWeights), c_void_p, c_void_p, c_int,
+                                         c_int, c_void_p, c_void_p, c_void_p]),
     "zi_model_forward": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "zi_euler_step": (c_int, [c_void_p, c_void_p, c_void_p, c_float, c_double, c_double, c_size_t, c_void_p]),

@@ -391,6 +391,29 @@ int run_rope(const zi_config& cfg, const int32_t* pos, int n, float2* out, cudaS
   return launched(ZI_KERNEL_ROPE, st);
 }
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch of zi_block_forward_noalloc: a file-scope device array, so the entry
+// point needs no caller workspace and allocates nothing.  Host code must not use
+// the symbol as a pointer (on the host it names a stand-in object, not device
+// memory); the device address is looked up once per device with that device
+// current and cached.
+static __device__ __align__(256) unsigned char g_zi_static_scratch[ZI_STATIC_SCRATCH_BYTES];
+
+void* g_scratch_addr[kMaxDevices] = {};
+
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZI_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_zi_static_scratch) != cudaSuccess || !p) return ZI_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return ZI_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -407,6 +430,7 @@ const char* zi_status_string(int s) {
     case ZI_ERR_CUDA: return "CUDA call failed";
     case ZI_ERR_TIMEOUT: return "device pipeline wait timed out";
     case ZI_ERR_DEVICE: return "current device is not an sm_100 GPU";
+    case ZI_ERR_SCRATCH_LIMIT: return "sizes exceed the library's fixed scratch (ZI_STATIC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }
@@ -606,6 +630,22 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   ZI_TRY(run_rms_mod<float>(d_x_in, rows, D, w->g_attn1, b.mod, b.mod_ld, b.map, 0, cfg->norm_eps, b.h, st));
   const NextNormSpec none{NEXT_NONE, nullptr, nullptr, 0};
   return run_block(b, none, st);
+}
+
+int zi_block_forward_noalloc(const zi_config* cfg, const zi_block_weights* w, const float* d_c,
+                             const int32_t* d_pos, int batch, int seq, const float* d_x_in, float* d_x_out,
+                             zi_stream_t stream) {
+  ZI_TRY(check_cfg(cfg));
+  if (batch <= 0 || seq <= 0) return ZI_ERR_ARG;
+  if (size_t(batch) * seq > (size_t(1) << 30)) return ZI_ERR_SHAPE;
+  if (carve(*cfg, batch, seq, 0, false, 4 * cfg->dim).total > size_t(ZI_STATIC_SCRATCH_BYTES))
+    return ZI_ERR_SCRATCH_LIMIT;
+  DevInfo* dev;
+  ZI_TRY(current_device(&dev));
+  void* ws = nullptr;
+  ZI_TRY(static_scratch(&ws));
+  return zi_block_forward(cfg, w, d_c, d_pos, batch, seq, d_x_in, d_x_out, ws, size_t(ZI_STATIC_SCRATCH_BYTES),
+                          stream);
 }
 
 int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
