@@ -392,6 +392,40 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     print(json.dumps(line), flush=True)
 
 
+def run_block_workload(args):
+    """One full-width main block over the 4,128-token sequence (profiling-sized case, < 1 GB on the device)."""
+    import torch
+
+    from stream_diffusion_transformer_b200 import abi, model
+
+    d = dataclasses.replace(zi.FULL, n_noise=0, n_ctx=0, n_main=1)
+    cfg = model.make_config(d)
+    gh, gw = LAT_H // 2, LAT_W // 2
+    S = gh * gw + S_TXT
+    bits = zi.make_weights(d, seed=SEED, keys=model.block_keys("layers.0", True), threads=8)
+    blk = model.DeviceBlock(cfg, "layers.0", bits, True, "cuda")
+    x = torch.from_numpy(zi.make_stream(d, 1, S, seed=SEED)).cuda()
+    c = torch.from_numpy(zi.make_cond(d, 1, seed=SEED)).cuda()
+    pos = model.positions(S_TXT, gh, gw)
+    out = torch.empty_like(x)
+    ws = torch.empty(abi.block_workspace_size(cfg, 1, S), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        model.block_forward(cfg, blk, c, pos, x, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with abi.Profile(capacity=16 * args.steps + 16) as prof:
+        e0.record()
+        for _ in range(args.steps):
+            model.block_forward(cfg, blk, c, pos, x, out, ws)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    fl = block_flops(S, d.dim, d.ffn)
+    print(json.dumps({"workload": f"one main block, full width, {S} tokens", "ms_per_step": ms,
+                      "value": fl / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "steps": args.steps,
+                      "kernels": prof.by_kernel(), "device_status": abi.device_status()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -399,7 +433,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["forward", "block"], default="forward",
+                    help="forward: the 4,128-token full forward (the metric); block: one main block of it "
+                         "(a profiling-sized case)")
     args = ap.parse_args()
+    if args.workload == "block":
+        run_block_workload(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
