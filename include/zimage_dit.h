@@ -76,8 +76,8 @@ typedef struct zi_config {
   int head_dim;     /* 128 (the only supported value) */
   int ffn;          /* SwiGLU inner width F (10240) */
   int cap_dim;      /* text-feature width (2560) */
-  int t_freq;       /* sinusoidal timestep width (256) */
-  int t_mid;        /* timestep MLP hidden width (1024) */
+  int t_freq;       /* sinusoidal timestep width (256, the only supported value) */
+  int t_mid;        /* timestep MLP hidden width (1024; multiple of 8) */
   int in_ch;        /* latent channels (16) */
   int patch;        /* 2 (the only supported value) */
   int n_noise;      /* noise-refiner blocks (2) */

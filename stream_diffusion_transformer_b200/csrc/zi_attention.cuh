@@ -217,14 +217,21 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&s_free[bi]);
 
-      float mx = -INFINITY;
+      // Row max and row sum use 8 independent chains each, so the per-element
+      // FMNMX / FFMA / EX2 / FADD of different columns overlap instead of
+      // waiting on one serial dependency chain.
+      if (kvn < 128) {  // the segment's last key tile: mask the columns past its end
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = __uint_as_float(s[c]);
-        if (c >= kvn) v = -INFINITY;
-        s[c] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < 128; ++c)
+          if (c >= kvn) s[c] = __float_as_uint(-INFINITY);
       }
+      float mxs[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mxs[k] = __uint_as_float(s[k]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mxs[c & 7] = fmaxf(mxs[c & 7], __uint_as_float(s[c]));
+      const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                             fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
       const float m_new = fmaxf(m_run, mx * sl2);
       const bool need = m_new > m_run + 8.0f;
       float alpha = 1.0f;
@@ -234,14 +241,17 @@ __global__ void __launch_bounds__(192, 1)
         m_run = m_new;
         l *= alpha;
       }
-      float sum = 0.f;
+      const float neg_m = -m_run;
+      float sums[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sums[k] = 0.f;
 #pragma unroll
       for (int c = 0; c < 128; ++c) {
-        const float e = fast_exp2(fmaf(__uint_as_float(s[c]), sl2, -m_run));
-        sum += e;
+        const float e = fast_exp2(fmaf(__uint_as_float(s[c]), sl2, neg_m));
+        sums[c & 7] += e;
         s[c] = __float_as_uint(e);
       }
-      l += sum;
+      l += ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
       if (j >= 1) {
         if (!mbar_wait(p_free, uint32_t(j - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) { ok = false; break; }
         tc_fence_after();

@@ -33,8 +33,9 @@ ZI_DEV void st_bf16x4(uint16_t* p, float4 v) {
   *reinterpret_cast<uint2*>(p) = u;
 }
 
-// h[row] = bf16( gain * x / sqrt(mean(x^2) + eps) * (1 + scale[batch(row)]) )
-// x is fp32 (TIn = float) or bf16 (TIn = uint16_t); scale may be null (no modulation).
+// h[row] = bf16( gain * x / sqrt(mean(x^2) + eps) * mscale[batch(row)] )
+// x is fp32 (TIn = float) or bf16 (TIn = uint16_t); mscale holds 1 + scale as the
+// adaLN kernel stores it, or is null (no modulation).
 template <typename TIn>
 __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restrict__ x, int D,
                                                               const uint16_t* __restrict__ gain,
@@ -67,10 +68,7 @@ __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restr
     if (i < nvec) {
       const float4 g = ld_bf16x4(gain + 4 * i);
       float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (sc) {
-        const float4 s = reinterpret_cast<const float4*>(sc)[i];
-        m = make_float4(1.f + s.x, 1.f + s.y, 1.f + s.z, 1.f + s.w);
-      }
+      if (sc) m = reinterpret_cast<const float4*>(sc)[i];
       st_bf16x4(h + size_t(row) * D + 4 * i,
                 make_float4(v[k].x * r * g.x * m.x, v[k].y * r * g.y * m.y, v[k].z * r * g.z * m.z,
                             v[k].w * r * g.w * m.w));
@@ -85,17 +83,18 @@ enum NextNorm : int { NEXT_NONE = 0, NEXT_RMS = 1, NEXT_LAYERNORM = 2 };
 //   x_out = x_in + gate * g_post * o / sqrt(mean(o^2) + eps)      (gate = tanh(raw) or 1)
 //   h     = g_next * x_out / sqrt(mean(x_out^2) + eps) * (1 + scale)     (NEXT_RMS)
 //   h     = (x_out - mean) / sqrt(var + eps_ln) * (1 + scale)            (NEXT_LAYERNORM)
+// tanh(raw) and 1 + scale come precomputed from the adaLN kernel.
 // h is written only for rows < next_rows.
 struct PostParams {
   const float* x_in;
   float* x_out;
   const uint16_t* o;
   const uint16_t* g_post;
-  const float* gate;  // raw adaLN gate [B][gate_ld] or null (gate = 1)
+  const float* gate;  // tanh(gate) [B][gate_ld] or null (gate = 1)
   int gate_ld;
   int next;
   const uint16_t* g_next;  // NEXT_RMS gain
-  const float* scale;      // [B][scale_ld] or null (no modulation)
+  const float* scale;      // 1 + scale [B][scale_ld] or null (no modulation)
   int scale_ld;
   int next_rows;
   uint16_t* h;
@@ -110,17 +109,22 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
   const int row = blockIdx.x;
   const int D = p.D, nvec = D >> 2;
   const int b = p.map.batch(row + p.row_off);
-  float4 v[kRowMaxVec];
+  float4 v[kRowMaxVec], xv[kRowMaxVec];
   float ss = 0.f;
+  // issue every load of the row (o and x) before the first reduction
 #pragma unroll
   for (int k = 0; k < kRowMaxVec; ++k) {
     const int i = threadIdx.x + k * kRowThreads;
     v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    xv[k] = v[k];
     if (i < nvec) {
       v[k] = ld_bf16x4(p.o + size_t(row) * D + 4 * i);
-      ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+      xv[k] = reinterpret_cast<const float4*>(p.x_in + size_t(row) * D)[i];
     }
   }
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k)
+    ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
   const float ro = rsqrtf(block_sum_128(ss, red) / float(D) + p.eps);
   const float* gt = p.gate ? p.gate + size_t(b) * p.gate_ld : nullptr;
   float s1 = 0.f, s2 = 0.f;
@@ -128,13 +132,10 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
   for (int k = 0; k < kRowMaxVec; ++k) {
     const int i = threadIdx.x + k * kRowThreads;
     if (i < nvec) {
-      const float4 x = reinterpret_cast<const float4*>(p.x_in + size_t(row) * D)[i];
+      const float4 x = xv[k];
       const float4 g = ld_bf16x4(p.g_post + 4 * i);
       float4 a = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (gt) {
-        const float4 r = reinterpret_cast<const float4*>(gt)[i];
-        a = make_float4(tanhf(r.x), tanhf(r.y), tanhf(r.z), tanhf(r.w));
-      }
+      if (gt) a = reinterpret_cast<const float4*>(gt)[i];
       float4 y;
       y.x = x.x + a.x * g.x * (v[k].x * ro);
       y.y = x.y + a.y * g.y * (v[k].y * ro);
@@ -172,10 +173,7 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
       float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
       if (p.next == NEXT_RMS) g = ld_bf16x4(p.g_next + 4 * i);
       float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (sc) {
-        const float4 s = reinterpret_cast<const float4*>(sc)[i];
-        m = make_float4(1.f + s.x, 1.f + s.y, 1.f + s.z, 1.f + s.w);
-      }
+      if (sc) m = reinterpret_cast<const float4*>(sc)[i];
       st_bf16x4(p.h + size_t(row) * D + 4 * i,
                 make_float4((v[k].x - mu) * r * g.x * m.x, (v[k].y - mu) * r * g.y * m.y,
                             (v[k].z - mu) * r * g.z * m.z, (v[k].w - mu) * r * g.w * m.w));
@@ -228,56 +226,82 @@ __global__ void rope_table_kernel(const int* __restrict__ pos, int n, int a0, in
   out[idx] = make_float2(float(c), float(s));
 }
 
-// Timestep conditioning for one batch element per CTA (256 threads):
-// e = [cos(1000 t f_k), sin(1000 t f_k)], f_k = 10000^(-k/128) (sinusoid in fp64);
-// c = W2 SiLU(W1 e + b1) + b2; also writes SiLU(c) for the final layer's adaLN.
-__global__ void __launch_bounds__(256) timestep_mlp_kernel(const float* __restrict__ t, float t_scale, int t_freq,
-                                                           int t_mid, int ada, const uint16_t* __restrict__ w1,
-                                                           const uint16_t* __restrict__ b1,
-                                                           const uint16_t* __restrict__ w2,
-                                                           const uint16_t* __restrict__ b2, float* __restrict__ c,
-                                                           float* __restrict__ silu_c) {
-  extern __shared__ float sh[];
-  float* e = sh;            // [t_freq]
-  float* hid = sh + t_freq; // [t_mid]
-  const int b = blockIdx.x;
-  const int half = t_freq / 2;
+// Timestep conditioning, step 1: hid[b] = SiLU(W1 e + b1) with
+// e = [cos(1000 t f_k), sin(1000 t f_k)], f_k = 10000^(-k/(t_freq/2)) (sinusoid in
+// fp64).  grid (t_mid / 8, B), 256 threads: each CTA rebuilds e in smem, one warp
+// per hidden unit with 16-byte weight loads (t_freq == 256: 8 inputs per lane).
+__global__ void __launch_bounds__(256) temb_hidden_kernel(const float* __restrict__ t, float t_scale, int t_mid,
+                                                          const uint16_t* __restrict__ w1,
+                                                          const uint16_t* __restrict__ b1, float* __restrict__ hid) {
+  __shared__ float e[256];
+  const int b = blockIdx.y;
   const double tin = double(t[b]) * double(t_scale);
-  for (int k = threadIdx.x; k < half; k += blockDim.x) {
-    const double f = exp(-log(10000.0) * double(k) / double(half));
-    double s, co;
-    sincos(tin * f, &s, &co);
+  for (int k = threadIdx.x; k < 128; k += blockDim.x) {
+    const double f = exp(-log(10000.0) * double(k) / 128.0);
+    double sn, co;
+    sincos(tin * f, &sn, &co);
     e[k] = float(co);
-    e[k + half] = float(s);
+    e[k + 128] = float(sn);
   }
   __syncthreads();
-  for (int o = threadIdx.x; o < t_mid; o += blockDim.x) {
-    float acc = bf16_to_f32(b1[o]);
-    const uint16_t* wr = w1 + size_t(o) * t_freq;
-    for (int i = 0; i < t_freq; ++i) acc = fmaf(bf16_to_f32(wr[i]), e[i], acc);
-    hid[o] = acc / (1.0f + expf(-acc));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o = blockIdx.x * 8 + warp;
+  if (o >= t_mid) return;
+  const uint4 wv = *reinterpret_cast<const uint4*>(w1 + size_t(o) * 256 + lane * 8);
+  const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    acc = fmaf(__uint_as_float(ww[q] << 16), e[lane * 8 + 2 * q], acc);
+    acc = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), e[lane * 8 + 2 * q + 1], acc);
   }
-  __syncthreads();
-  for (int o = threadIdx.x; o < ada; o += blockDim.x) {
-    float acc = bf16_to_f32(b2[o]);
-    const uint16_t* wr = w2 + size_t(o) * t_mid;
-    for (int i = 0; i < t_mid; ++i) acc = fmaf(bf16_to_f32(wr[i]), hid[i], acc);
+  acc = warp_sum(acc) + bf16_to_f32(b1[o]);
+  if (lane == 0) hid[size_t(b) * t_mid + o] = acc / (1.0f + expf(-acc));
+}
+
+// Timestep conditioning, step 2: c[b] = W2 hid[b] + b2 (and SiLU(c) for the final
+// layer's adaLN).  grid (ada / 8, B), one warp per output, 16-byte weight loads.
+__global__ void __launch_bounds__(256) temb_out_kernel(const float* __restrict__ hid, int t_mid, int ada,
+                                                       const uint16_t* __restrict__ w2,
+                                                       const uint16_t* __restrict__ b2, float* __restrict__ c,
+                                                       float* __restrict__ silu_c) {
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o = blockIdx.x * 8 + warp;
+  if (o >= ada) return;
+  const uint16_t* wr = w2 + size_t(o) * t_mid;
+  const float* h = hid + size_t(b) * t_mid;
+  float acc = 0.f;
+  for (int i = lane * 8; i < t_mid; i += 256) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(wr + i);
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc = fmaf(__uint_as_float(ww[q] << 16), h[i + 2 * q], acc);
+      acc = fmaf(__uint_as_float(ww[q] & 0xFFFF0000u), h[i + 2 * q + 1], acc);
+    }
+  }
+  acc = warp_sum(acc) + bf16_to_f32(b2[o]);
+  if (lane == 0) {
     c[size_t(b) * ada + o] = acc;
     silu_c[size_t(b) * ada + o] = acc / (1.0f + expf(-acc));
   }
 }
 
-// All adaLN projections of a forward in one launch: segment s maps its input
-// vector (c, or SiLU(c) for the final layer) through w_s [rows_s, 256] + b_s into
-// out[b][off_s + row].  One warp per output row, 16-byte weight loads.
+// All adaLN projections of a forward in one launch, stored as the factors the
+// row kernels multiply by.  A block segment (4D rows: scale_msa, gate_msa,
+// scale_mlp, gate_mlp) maps c through w_s + b_s and stores 1 + scale and
+// tanh(gate); the final layer's segment (D rows) maps SiLU(c) and stores
+// 1 + scale.  out[b][off_s + row].  One warp per output row, 16-byte weight loads.
 constexpr int kMaxAdaSegs = 40;
 struct AdaSegs {
   const uint16_t* w[kMaxAdaSegs];
   const uint16_t* b[kMaxAdaSegs];
   int rows[kMaxAdaSegs];
   int off[kMaxAdaSegs];
-  int silu[kMaxAdaSegs];
+  int final_seg[kMaxAdaSegs];  // 1: input SiLU(c), all rows are scales; 0: a block's 4 bands
   int n;
+  int dim;
 };
 
 __global__ void __launch_bounds__(256) ada_gemv_kernel(AdaSegs segs, const float* __restrict__ c,
@@ -287,7 +311,8 @@ __global__ void __launch_bounds__(256) ada_gemv_kernel(AdaSegs segs, const float
   const int s = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = segs.rows[s];
-  const float* in = segs.silu[s] ? silu_c : c;
+  const bool fin = segs.final_seg[s] != 0;
+  const float* in = fin ? silu_c : c;
   for (int r = blockIdx.x * 8 + warp; r < rows; r += gridDim.x * 8) {
     const uint4 wv = *reinterpret_cast<const uint4*>(segs.w[s] + size_t(r) * 256 + lane * 8);
     const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -298,13 +323,14 @@ __global__ void __launch_bounds__(256) ada_gemv_kernel(AdaSegs segs, const float
       wf[2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
     }
     const float bias = bf16_to_f32(segs.b[s][r]);
+    const bool is_gate = !fin && ((r / segs.dim) & 1);  // bands 1 and 3 of a block are gates
     for (int b = 0; b < batch; ++b) {
       const float4 i0 = *reinterpret_cast<const float4*>(in + size_t(b) * 256 + lane * 8);
       const float4 i1 = *reinterpret_cast<const float4*>(in + size_t(b) * 256 + lane * 8 + 4);
       float acc = wf[0] * i0.x + wf[1] * i0.y + wf[2] * i0.z + wf[3] * i0.w + wf[4] * i1.x + wf[5] * i1.y +
                   wf[6] * i1.z + wf[7] * i1.w;
-      acc = warp_sum(acc);
-      if (lane == 0) out[size_t(b) * out_ld + segs.off[s] + r] = acc + bias;
+      acc = warp_sum(acc) + bias;
+      if (lane == 0) out[size_t(b) * out_ld + segs.off[s] + r] = is_gate ? tanhf(acc) : 1.0f + acc;
     }
   }
 }

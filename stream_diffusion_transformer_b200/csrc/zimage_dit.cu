@@ -233,7 +233,7 @@ constexpr size_t kAlign = 1024;
 inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-  size_t mod, c, silu, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
+  size_t mod, c, silu, hid, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
 };
 
 Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int mod_cols) {
@@ -247,6 +247,7 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.mod = o; o = up(o + size_t(batch) * size_t(mod_cols) * 4);
   w.c = o; o = up(o + (model ? size_t(batch) * 256 * 4 : 0));
   w.silu = o; o = up(o + (model ? size_t(batch) * 256 * 4 : 0));
+  w.hid = o; o = up(o + (model ? size_t(batch) * size_t(cfg.t_mid) * 4 : 0));
   w.pos = o; o = up(o + (model ? S * 3 * 4 : 0));
   w.rope = o; o = up(o + S * pairs * 8);
   w.x = o; o = up(o + (model ? rows * D * 4 : 0));
@@ -269,7 +270,7 @@ int check_cfg(const zi_config* c) {
   for (int i = 0; i < 3; ++i)
     if (c->rope_axes[i] <= 0 || c->rope_axes[i] % 2) return ZI_ERR_SHAPE;
   if (c->ffn <= 0 || c->cap_dim <= 0 || c->cap_dim % 64 != 0 || c->cap_dim > 4096) return ZI_ERR_SHAPE;
-  if (c->t_freq <= 0 || c->t_freq % 2 || c->t_mid <= 0) return ZI_ERR_SHAPE;
+  if (c->t_freq != 256 || c->t_mid <= 0 || c->t_mid % 8) return ZI_ERR_SHAPE;  // warp-per-row timestep MLP
   if ((c->dim < 256 ? c->dim : 256) != 256) return ZI_ERR_SHAPE;  // adaLN GEMV is 256 wide
   if (4 * c->in_ch != 64) return ZI_ERR_SHAPE;                     // final linear uses a 64-wide tile
   if (c->n_noise < 0 || c->n_ctx < 0 || c->n_main < 1 || c->n_noise + c->n_main + 1 > kMaxAdaSegs)
@@ -599,7 +600,7 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
     segs.b[0] = w->b_ada;
     segs.rows[0] = 4 * D;
     segs.off[0] = 0;
-    segs.silu[0] = 0;
+    segs.dim = D;
     ZI_TRY(run_ada(segs, d_c, d_c, batch, 4 * D, mod, st));
   }
   ZI_TRY(run_rope(*cfg, d_pos, seq, rope, st));
@@ -704,11 +705,13 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
 
   // timestep conditioning and every adaLN projection
   {
-    const int smem = (cfg->t_freq + cfg->t_mid) * 4;
-    if (smem > 48 * 1024) return ZI_ERR_SHAPE;
+    float* hid = reinterpret_cast<float*>(ws + L.hid);
     prof_pre(st);
-    timestep_mlp_kernel<<<batch, 256, smem, st>>>(d_t, cfg->t_scale, cfg->t_freq, cfg->t_mid, 256, w->t_w1,
-                                                  w->t_b1, w->t_w2, w->t_b2, c, silu_c);
+    temb_hidden_kernel<<<dim3((cfg->t_mid + 7) / 8, batch), 256, 0, st>>>(d_t, cfg->t_scale, cfg->t_mid, w->t_w1,
+                                                                         w->t_b1, hid);
+    ZI_TRY(launched(ZI_KERNEL_TIMESTEP, st));
+    prof_pre(st);
+    temb_out_kernel<<<dim3(256 / 8, batch), 256, 0, st>>>(hid, cfg->t_mid, 256, w->t_w2, w->t_b2, c, silu_c);
     ZI_TRY(launched(ZI_KERNEL_TIMESTEP, st));
     AdaSegs segs;
     memset(&segs, 0, sizeof(segs));
@@ -729,8 +732,9 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
     segs.b[k] = w->final_ada_b;
     segs.rows[k] = D;
     segs.off[k] = n_mod * 4 * D;
-    segs.silu[k] = 1;
+    segs.final_seg[k] = 1;
     segs.n = k + 1;
+    segs.dim = D;
     ZI_TRY(run_ada(segs, c, silu_c, batch, mod_ld, mod, st));
   }
   auto mod_of_noise = [&](int i) { return mod + size_t(i) * 4 * D; };
