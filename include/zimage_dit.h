@@ -214,9 +214,9 @@ ZI_API int zi_sigmas(int n_steps, double shift, double* h_sigmas);
  * cudaMalloc after start-up (cudaMalloc can synchronise the device and stall
  * other work).  Such callers cannot provide the workspace zi_block_forward needs. */
 
-/* Bytes of the library's fixed device scratch (64 MiB).  Every GPU that loads the
+/* Bytes of the library's fixed device scratch (128 MiB).  Every GPU that loads the
  * library holds this much device memory until the process exits. */
-#define ZI_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+#define ZI_STATIC_SCRATCH_BYTES (128u * 1024u * 1024u)
 
 /* zi_block_forward without a workspace argument: the scratch is a file-scope
  * device array of ZI_STATIC_SCRATCH_BYTES inside the library.  The caller still
@@ -224,7 +224,7 @@ ZI_API int zi_sigmas(int n_steps, double shift, double* h_sigmas);
  * for zi_block_forward.
  *   - Allocates nothing: no cudaMalloc/cudaFree and no allocating library call.
  *   - Sizes whose zi_block_workspace_size() exceeds ZI_STATIC_SCRATCH_BYTES are
- *     rejected with ZI_ERR_SCRATCH_LIMIT before anything is enqueued (about 990
+ *     rejected with ZI_ERR_SCRATCH_LIMIT before anything is enqueued (about 1,350
  *     tokens of batch x seq at Z-Image's full width).
  *   - The first call on each device looks up the scratch's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
@@ -251,9 +251,17 @@ ZI_API int zi_positions(int s_txt, int grid_h, int grid_w, int32_t* d_pos, zi_st
  * pos[axis] * theta^(-2j/d_axis) for rotation pair j (pairs of axis 0 first). */
 ZI_API int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, float* d_cos_sin, zi_stream_t stream);
 
+/* Bytes of split scratch zi_gemm_bf16 can use (about 42 MB). */
+ZI_API int zi_gemm_workspace_size(size_t* h_bytes);
+
 /* C[M, N] = A[M, K] B[N, K]^T, bf16 in, fp32 accumulate, bf16 out (tcgen05).
- * K % 64 == 0, N % 256 == 0, M >= 1; rows are contiguous (strides K and N). */
-ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, zi_stream_t stream);
+ * K % 64 == 0, N % 256 == 0, M >= 1; rows are contiguous (strides K and N).
+ * d_ws (256-byte aligned, >= zi_gemm_workspace_size() bytes) may be NULL; when
+ * given, the tiles of the ragged last wave are split along K over all SMs
+ * (stream-K) instead of leaving SMs idle; the result is the same up to fp32
+ * summation order. */
+ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, void* d_ws,
+                        size_t ws_bytes, zi_stream_t stream);
 
 /* Non-causal softmax(q k^T / sqrt(128)) v per head over seq tokens per batch element.
  * d_qkv bf16 [batch*seq, 3*heads*128] (q | k | v, head h at columns h*128 of each);

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzimage_d
 ZI_OK, ZI_ERR_ARG, ZI_ERR_SHAPE, ZI_ERR_ALIGN, ZI_ERR_WORKSPACE, ZI_ERR_CUDA, ZI_ERR_TIMEOUT, ZI_ERR_DEVICE = (
     0, -1, -2, -3, -4, -5, -6, -7)
 ZI_ERR_SCRATCH_LIMIT = -8
-STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
+STATIC_SCRATCH_BYTES = 128 * 1024 * 1024
 
 
 class ZiError(RuntimeError):
@@ -69,7 +69,8 @@ _SIGS = {
     "zi_sigmas": (c_int, [c_int, c_double, POINTER(c_double)]),
     "zi_positions": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
-    "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_gemm_workspace_size": (c_int, [POINTER(c_size_t)]),
+    "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_profile_begin": (c_int, [c_int]),
     "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),

@@ -56,7 +56,7 @@ struct GemmSmem {
   static constexpr uint32_t kBBytes = uint32_t(BN) * 64u * 2u;
   static constexpr uint32_t kStage = kABytes + kBBytes;
   static constexpr uint32_t kBarOff = STAGES * kStage;
-  static constexpr uint32_t kBytes = kBarOff + 256u + 1024u;  // + barriers + alignment slack
+  static constexpr uint32_t kBytes = kBarOff + 256u + 1024u;  // + barriers/flags (< 256 B) + alignment slack
   static constexpr uint32_t kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                         : (2 * BN <= 256) ? 256 : 512;
 };
@@ -201,10 +201,94 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const Ep
   }
 }
 
+// Work schedule: data-parallel tiles first, then a stream-K tail.
+//
+// With T output tiles on G persistent CTAs, T % G != 0 leaves a ragged last
+// wave.  When the caller provides split scratch, the last (G + T % G) tiles are
+// instead cut into k-block units spread evenly over all G CTAs (each CTA gets
+// one contiguous run of units, crossing tile boundaries).  A tile covered by
+// several CTAs is finished by whichever contributor arrives last: every
+// contributor stores its fp32 partial in its own scratch slot and bumps the
+// tile's counter; the CTA that completes the count adds the other partials
+// into its accumulator and runs the fused epilogue.  Nobody waits on another
+// CTA, so the schedule needs no co-residency.
+struct SkSched {
+  int tiles;     // T
+  int grid;      // G (persistent CTAs)
+  int kb;        // k-blocks per tile
+  int dp_tiles;  // tiles [0, dp_tiles) are whole-tile work, walked with stride G
+  int base, rem; // stream-K units per CTA: base (+1 for the first rem CTAs)
+  __host__ __device__ int unit_begin(int c) const { return c * base + (c < rem ? c : rem); }
+  __host__ __device__ int cta_of_unit(int u) const {
+    const int big = rem * (base + 1);
+    return u < big ? u / (base + 1) : rem + (u - big) / base;
+  }
+};
+
+inline SkSched make_sk_sched(int tiles, int grid, int kb, bool split) {
+  SkSched s;
+  s.tiles = tiles;
+  s.grid = grid;
+  s.kb = kb;
+  s.dp_tiles = tiles;
+  s.base = 0;
+  s.rem = 0;
+  if (split && tiles > grid && tiles % grid != 0) {
+    s.dp_tiles = (tiles / grid - 1) * grid;
+    const long long units = static_cast<long long>(tiles - s.dp_tiles) * kb;
+    s.base = static_cast<int>(units / grid);
+    s.rem = static_cast<int>(units % grid);
+  }
+  return s;
+}
+
+struct WorkItem {
+  int tile, kb0, kb1;
+  int sk_tile;  // -1: the whole tile is this CTA's; else index of the split tile
+  int slot;     // scratch slot of this CTA's partial (2c for its first run, 2c + 1 for its last)
+};
+
+// Walks one CTA's work items; every warp role walks the same sequence.
+struct WorkWalker {
+  const SkSched& s;
+  int c, next_dp, u, u0, u1;
+  ZI_DEV WorkWalker(const SkSched& sched, int cta)
+      : s(sched), c(cta), next_dp(cta), u0(sched.base ? sched.unit_begin(cta) : 0),
+        u1(sched.base ? sched.unit_begin(cta + 1) : 0) {
+    u = u0;
+  }
+  ZI_DEV bool next(WorkItem& w) {
+    if (next_dp < s.dp_tiles) {
+      w.tile = next_dp;
+      w.kb0 = 0;
+      w.kb1 = s.kb;
+      w.sk_tile = -1;
+      w.slot = -1;
+      next_dp += s.grid;
+      return true;
+    }
+    if (u >= u1) return false;
+    const int st = u / s.kb, k0 = u % s.kb;
+    const int k1 = min(s.kb, k0 + (u1 - u));
+    w.tile = s.dp_tiles + st;
+    w.kb0 = k0;
+    w.kb1 = k1;
+    w.sk_tile = (k0 == 0 && k1 == s.kb) ? -1 : st;
+    w.slot = (u == u0) ? 2 * c : 2 * c + 1;
+    u += k1 - k0;
+    return true;
+  }
+};
+
+struct SplitScratch {
+  float* partials;  // [2 * G][128 * BN] fp32 (row-major, the accumulator tile as is)
+  int* counters;    // [max split tiles], zero on entry; reset to zero by each tile's finisher
+};
+
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                        int N, int K, EpiParams ep) {
+                        int N, int K, EpiParams ep, SkSched sched, SplitScratch sk) {
   using L = GemmSmem<BN, STAGES>;
   constexpr int BM = 128, BK = 64;
   extern __shared__ uint8_t smem_raw[];
@@ -214,8 +298,10 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ebar = drain + 1;  // syncs the 128 epilogue threads (bounded wait, unlike bar.sync)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
 
   if (device_error_set()) return;  // an earlier kernel timed out: leave everything untouched
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,6 +316,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(ebar, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -247,16 +334,16 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_m = (M + BM - 1) / BM;
-  const int num_tiles = num_m * (N / BN);
-  const int KB = K / BK;
+  WorkItem wi;
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
-        for (int kb = 0; kb < KB; ++kb) {
+      WorkWalker walk(sched, blockIdx.x);
+      while (ok && walk.next(wi)) {
+        const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) {
             ok = false;
@@ -285,16 +372,18 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       int local = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      WorkWalker walk(sched, blockIdx.x);
+      while (ok && walk.next(wi)) {
         const int acc = local & 1;
         const uint32_t u = uint32_t(local) >> 1;
+        ++local;
         if (!mbar_wait(&tempty[acc], (u & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&full[s], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
             ok = false;
@@ -306,7 +395,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             tc_mma(d, smem_desc_sw128(a_addr + k * 32, 16), smem_desc_sw128(b_addr + k * 32, 16), idesc,
-                   (kb | k) != 0 ? 1u : 0u);
+                   (kb > wi.kb0 || k > 0) ? 1u : 0u);
           }
           tc_commit(&empty[s]);
           ++it;
@@ -324,15 +413,73 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;  // this warp's TMEM lane quarter
     const int row_in_tile = q * 32 + lane;
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    uint32_t ephase = 0;
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(ebar);
+      const bool r = mbar_wait(ebar, ephase, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE);
+      ephase ^= 1u;
+      return r;
+    };
+    WorkWalker walk(sched, blockIdx.x);
+    while (walk.next(wi)) {
       const int acc = local & 1;
       const uint32_t u = uint32_t(local) >> 1;
+      ++local;
       if (!mbar_wait(&tfull[acc], u & 1u, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+      const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
       const int row = m0 + row_in_tile;
       const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-      gemm_epilogue<EPI, BN>(tb, row, row < M, n0, ep);
+      bool finish = true;
+      if (wi.sk_tile >= 0) {
+        // Split tile: publish this CTA's partial, and finish the tile only if last.
+        float* mine = sk.partials + size_t(wi.slot) * (128 * BN) + size_t(row_in_tile) * BN;
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(tb + c * 32, v);
+          float4* d4 = reinterpret_cast<float4*>(mine + c * 32);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            __stcg(d4 + k, make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+        }
+        __threadfence();
+        if (!epi_sync()) break;
+        const int t0u = wi.sk_tile * sched.kb;
+        const int c_lo = sched.cta_of_unit(t0u), c_hi = sched.cta_of_unit(t0u + sched.kb - 1);
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(&sk.counters[wi.sk_tile], 1);
+          const bool last = old == c_hi - c_lo;
+          if (last) sk.counters[wi.sk_tile] = 0;  // ready for the next launch
+          *last_flag = last ? 1 : 0;
+        }
+        if (!epi_sync()) break;
+        finish = *last_flag != 0;
+        if (finish) {
+          __threadfence();
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32_sync(tb + c * 32, v);
+            for (int cc = c_lo; cc <= c_hi; ++cc) {
+              const int slot = sched.unit_begin(cc) >= t0u ? 2 * cc : 2 * cc + 1;
+              if (slot == wi.slot) continue;
+              const float4* p4 = reinterpret_cast<const float4*>(sk.partials + size_t(slot) * (128 * BN) +
+                                                                 size_t(row_in_tile) * BN + c * 32);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float4 a = __ldcg(p4 + k);
+                v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + a.x);
+                v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + a.y);
+                v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + a.z);
+                v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + a.w);
+              }
+            }
+            tmem_st32(tb + c * 32, v);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (finish) gemm_epilogue<EPI, BN>(tb, row, row < M, n0, ep);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

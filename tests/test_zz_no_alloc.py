@@ -3,7 +3,7 @@
 Some callers cannot hand the library a workspace: a plugin inside a host
 program whose memory manager owns all device memory and gives plugins no
 allocator, or a latency-critical loop that forbids cudaMalloc after start-up.
-For them the library keeps a fixed 64 MiB device scratch array of its own.
+For them the library keeps a fixed 128 MiB device scratch array of its own.
 This test calls that entry point through the C ABI twice in a row (different
 inputs, so the second call runs on scratch the first one left behind) and
 checks each result against zi_block_forward given a freshly allocated
