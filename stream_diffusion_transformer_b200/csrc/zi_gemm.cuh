@@ -248,7 +248,9 @@ struct WorkItem {
   int slot;     // scratch slot of this CTA's partial (2c for its first run, 2c + 1 for its last)
 };
 
-// Walks one CTA's work items; every warp role walks the same sequence.
+// Walks one CTA's work items; every warp role walks the same sequence.  The
+// stream-K run comes first, so the fix-up of split tiles (reading the other
+// contributors' partials) overlaps the main loops of the whole tiles that follow.
 struct WorkWalker {
   const SkSched& s;
   int c, next_dp, u, u0, u1;
@@ -258,6 +260,17 @@ struct WorkWalker {
     u = u0;
   }
   ZI_DEV bool next(WorkItem& w) {
+    if (u < u1) {
+      const int st = u / s.kb, k0 = u % s.kb;
+      const int k1 = min(s.kb, k0 + (u1 - u));
+      w.tile = s.dp_tiles + st;
+      w.kb0 = k0;
+      w.kb1 = k1;
+      w.sk_tile = (k0 == 0 && k1 == s.kb) ? -1 : st;
+      w.slot = (u == u0) ? 2 * c : 2 * c + 1;
+      u += k1 - k0;
+      return true;
+    }
     if (next_dp < s.dp_tiles) {
       w.tile = next_dp;
       w.kb0 = 0;
@@ -267,16 +280,7 @@ struct WorkWalker {
       next_dp += s.grid;
       return true;
     }
-    if (u >= u1) return false;
-    const int st = u / s.kb, k0 = u % s.kb;
-    const int k1 = min(s.kb, k0 + (u1 - u));
-    w.tile = s.dp_tiles + st;
-    w.kb0 = k0;
-    w.kb1 = k1;
-    w.sk_tile = (k0 == 0 && k1 == s.kb) ? -1 : st;
-    w.slot = (u == u0) ? 2 * c : 2 * c + 1;
-    u += k1 - k0;
-    return true;
+    return false;
   }
 };
 
@@ -458,21 +462,27 @@ __global__ void __launch_bounds__(192, 1)
         if (finish) {
           __threadfence();
           for (int c = 0; c < BN / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32_sync(tb + c * 32, v);
+            // The other contributor's partial for these 32 columns.  Every CTA's run is
+            // at least kb units long (the split part holds more than G tiles), so at
+            // most two runs meet in one tile: there is exactly one other partial.
+            int other = -1;
             for (int cc = c_lo; cc <= c_hi; ++cc) {
               const int slot = sched.unit_begin(cc) >= t0u ? 2 * cc : 2 * cc + 1;
-              if (slot == wi.slot) continue;
-              const float4* p4 = reinterpret_cast<const float4*>(sk.partials + size_t(slot) * (128 * BN) +
-                                                                 size_t(row_in_tile) * BN + c * 32);
+              if (slot != wi.slot) other = slot;
+            }
+            float4 pa[8];
+            const float4* p4 = reinterpret_cast<const float4*>(sk.partials + size_t(other < 0 ? wi.slot : other) *
+                                                               (128 * BN) + size_t(row_in_tile) * BN + c * 32);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const float4 a = __ldcg(p4 + k);
-                v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + a.x);
-                v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + a.y);
-                v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + a.z);
-                v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + a.w);
-              }
+            for (int k = 0; k < 8; ++k) pa[k] = other < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(p4 + k);
+            uint32_t v[32];
+            tmem_ld32_sync(tb + c * 32, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + pa[k].x);
+              v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + pa[k].y);
+              v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + pa[k].z);
+              v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + pa[k].w);
             }
             tmem_st32(tb + c * 32, v);
           }

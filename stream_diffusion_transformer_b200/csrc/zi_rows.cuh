@@ -1,23 +1,26 @@
 // Bandwidth-bound kernels: row norms with modulation and gated residuals,
 // positions and the RoPE table, the timestep MLP, the batched adaLN GEMV,
 // patchify, and the Euler / CFG step.  One CTA per row for the row kernels
-// (128 threads, float4 / 8-byte bf16 vectors, every byte read once).
+// (256 threads, float4 / 8-byte bf16 vectors, every byte read once).
 #pragma once
 #include "zi_common.cuh"
 #include "zi_gemm.cuh"
 
 namespace zi {
 
-constexpr int kRowThreads = 128;
-constexpr int kRowMaxVec = 8;  // float4 per thread: rows up to 128 * 8 * 4 = 4096 wide
+constexpr int kRowThreads = 256;
+constexpr int kRowMaxVec = 4;  // float4 per thread: rows up to 256 * 4 * 4 = 4096 wide
 
-ZI_DEV float block_sum_128(float v, float* red) {
+ZI_DEV float block_sum(float v, float* red) {
   v = warp_sum(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   __syncthreads();  // `red` may still be read from a previous reduction
   if (l == 0) red[w] = v;
   __syncthreads();
-  return red[0] + red[1] + red[2] + red[3];
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRowThreads / 32; ++i) t += red[i];
+  return t;
 }
 
 ZI_DEV float4 ld_bf16x4(const uint16_t* p) {
@@ -42,7 +45,7 @@ __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restr
                                                               const float* __restrict__ scale, int scale_ld,
                                                               RowMap map, int row_off, float eps,
                                                               uint16_t* __restrict__ h) {
-  __shared__ float red[4];
+  __shared__ float red[kRowThreads / 32];
   const int row = blockIdx.x;
   const int nvec = D >> 2;
   float4 v[kRowMaxVec];
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restr
       ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
     }
   }
-  const float r = rsqrtf(block_sum_128(ss, red) / float(D) + eps);
+  const float r = rsqrtf(block_sum(ss, red) / float(D) + eps);
   const float* sc = scale ? scale + size_t(map.batch(row + row_off)) * scale_ld : nullptr;
 #pragma unroll
   for (int k = 0; k < kRowMaxVec; ++k) {
@@ -105,7 +108,7 @@ struct PostParams {
 };
 
 __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p) {
-  __shared__ float red[4];
+  __shared__ float red[kRowThreads / 32];
   const int row = blockIdx.x;
   const int D = p.D, nvec = D >> 2;
   const int b = p.map.batch(row + p.row_off);
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
 #pragma unroll
   for (int k = 0; k < kRowMaxVec; ++k)
     ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
-  const float ro = rsqrtf(block_sum_128(ss, red) / float(D) + p.eps);
+  const float ro = rsqrtf(block_sum(ss, red) / float(D) + p.eps);
   const float* gt = p.gate ? p.gate + size_t(b) * p.gate_ld : nullptr;
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll
@@ -150,9 +153,9 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
   if (p.next == NEXT_NONE || row >= p.next_rows) return;
   float mu = 0.f, r;
   if (p.next == NEXT_RMS) {
-    r = rsqrtf(block_sum_128(s2, red) / float(D) + p.eps);
+    r = rsqrtf(block_sum(s2, red) / float(D) + p.eps);
   } else {
-    mu = block_sum_128(s1, red) / float(D);
+    mu = block_sum(s1, red) / float(D);
     // variance from the centred values (second pass over registers)
     float sc = 0.f;
 #pragma unroll
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
         sc += a * a + bq * bq + c * c + d * d;
       }
     }
-    r = rsqrtf(block_sum_128(sc, red) / float(D) + p.eps_ln);
+    r = rsqrtf(block_sum(sc, red) / float(D) + p.eps_ln);
   }
   const float* sc = p.scale ? p.scale + size_t(b) * p.scale_ld : nullptr;
 #pragma unroll
