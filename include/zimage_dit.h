@@ -251,17 +251,13 @@ ZI_API int zi_positions(int s_txt, int grid_h, int grid_w, int32_t* d_pos, zi_st
  * pos[axis] * theta^(-2j/d_axis) for rotation pair j (pairs of axis 0 first). */
 ZI_API int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, float* d_cos_sin, zi_stream_t stream);
 
-/* Bytes of split scratch zi_gemm_bf16 can use (about 42 MB). */
-ZI_API int zi_gemm_workspace_size(size_t* h_bytes);
-
 /* C[M, N] = A[M, K] B[N, K]^T, bf16 in, fp32 accumulate, bf16 out (tcgen05).
  * K % 64 == 0, N % 256 == 0, M >= 1; rows are contiguous (strides K and N).
- * d_ws (256-byte aligned, >= zi_gemm_workspace_size() bytes) may be NULL; when
- * given, the tiles of the ragged last wave are split along K over all SMs
- * (stream-K) instead of leaving SMs idle; the result is the same up to fp32
- * summation order. */
-ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, void* d_ws,
-                        size_t ws_bytes, zi_stream_t stream);
+ * Same kernel and schedule as the projections of the forward: 128 x 256 tiles
+ * on persistent CTAs, a ragged last wave cut along N into 128 x 128 or 128 x 64
+ * sub-tiles. */
+ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k,
+                        zi_stream_t stream);
 
 /* Non-causal softmax(q k^T / sqrt(128)) v per head over seq tokens per batch element.
  * d_qkv bf16 [batch*seq, 3*heads*128] (q | k | v, head h at columns h*128 of each);

@@ -69,8 +69,7 @@ _SIGS = {
     "zi_sigmas": (c_int, [c_int, c_double, POINTER(c_double)]),
     "zi_positions": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
-    "zi_gemm_workspace_size": (c_int, [POINTER(c_size_t)]),
-    "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_profile_begin": (c_int, [c_int]),
     "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),

@@ -75,13 +75,15 @@ ZI_DEV void store_bf16x32(uint16_t* dst, const float* v) {
   }
 }
 
+// Epilogue of one tile of `width` columns (width <= BN, a multiple of 64)
+// starting at output column n0.
 template <int EPI, int BN>
-ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const EpiParams& ep) {
+ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int width, const EpiParams& ep) {
   uint32_t v[32];
   float f[32];
   if constexpr (EPI == EPI_BF16 || EPI == EPI_F32_BIAS) {
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 0; c < width / 32; ++c) {
       tmem_ld32_sync(tbase + c * 32, v);
       if (row_ok) {
         const int col = n0 + c * 32;
@@ -110,12 +112,12 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const Ep
       }
     }
   } else if constexpr (EPI == EPI_QKV) {
-    static_assert(BN == 256, "QKV epilogue works on two 128-wide heads per tile");
+    static_assert(BN == 256, "QKV epilogue works on 128-wide heads (two per full tile)");
     const int region = n0 / ep.dim;  // 0 = q, 1 = k, 2 = v
     uint16_t* orow = static_cast<uint16_t*>(ep.out) + size_t(row) * ep.ldo;
     if (region == 2) {
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < width / 32; ++c) {
         tmem_ld32_sync(tbase + c * 32, v);
         if (row_ok) {
 #pragma unroll
@@ -129,7 +131,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const Ep
     const int p = row_ok ? ep.map.pos(row + ep.row_off) : 0;
     const float2* rp = ep.rope + size_t(p) * 64;
 #pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {
+    for (int hh = 0; hh < width / 128; ++hh) {
       float ss = 0.f;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -185,7 +187,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const Ep
     const int b = gr / ep.s_img, t = gr % ep.s_img;
     const int ty = t / ep.grid_w, tx = t % ep.grid_w;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = 0; c < width / 32; ++c) {
       tmem_ld32_sync(tbase + c * 32, v);
       if (row_ok) {
 #pragma unroll 4
@@ -201,98 +203,71 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, const Ep
   }
 }
 
-// Work schedule: data-parallel tiles first, then a stream-K tail.
-//
-// With T output tiles on G persistent CTAs, T % G != 0 leaves a ragged last
-// wave.  When the caller provides split scratch, the last (G + T % G) tiles are
-// instead cut into k-block units spread evenly over all G CTAs (each CTA gets
-// one contiguous run of units, crossing tile boundaries).  A tile covered by
-// several CTAs is finished by whichever contributor arrives last: every
-// contributor stores its fp32 partial in its own scratch slot and bumps the
-// tile's counter; the CTA that completes the count adds the other partials
-// into its accumulator and runs the fused epilogue.  Nobody waits on another
-// CTA, so the schedule needs no co-residency.
-struct SkSched {
-  int tiles;     // T
-  int grid;      // G (persistent CTAs)
-  int kb;        // k-blocks per tile
-  int dp_tiles;  // tiles [0, dp_tiles) are whole-tile work, walked with stride G
-  int base, rem; // stream-K units per CTA: base (+1 for the first rem CTAs)
-  __host__ __device__ int unit_begin(int c) const { return c * base + (c < rem ? c : rem); }
-  __host__ __device__ int cta_of_unit(int u) const {
-    const int big = rem * (base + 1);
-    return u < big ? u / (base + 1) : rem + (u - big) / base;
-  }
+// Work schedule.  T output tiles of 128 x BN run on G persistent CTAs, tile t
+// on CTA t % G.  When T % G leaves a last wave of R < G tiles, and f R <= G for
+// a split factor f in {2, 4} the epilogue allows, those R tiles are cut along N
+// into f sub-tiles of BN / f columns each, one per CTA: the ragged wave then
+// costs 1/f of a tile's time instead of a whole one, with no reduction across
+// CTAs.
+struct TailSched {
+  int grid;        // G
+  int dp_tiles;    // tiles [0, dp_tiles) run whole, walked with stride G
+  int tail_f;      // sub-tiles per tail tile (1 = no tail)
+  int tail_items;  // CTAs [0, tail_items) each run one sub-tile of tile dp_tiles + c / tail_f
 };
 
-inline SkSched make_sk_sched(int tiles, int grid, int kb, bool split) {
-  SkSched s;
-  s.tiles = tiles;
-  s.grid = grid;
-  s.kb = kb;
-  s.dp_tiles = tiles;
-  s.base = 0;
-  s.rem = 0;
-  if (split && tiles > grid && tiles % grid != 0) {
-    s.dp_tiles = (tiles / grid - 1) * grid;
-    const long long units = static_cast<long long>(tiles - s.dp_tiles) * kb;
-    s.base = static_cast<int>(units / grid);
-    s.rem = static_cast<int>(units % grid);
+inline TailSched make_tail_sched(int tiles, int grid, int max_f) {
+  TailSched s{grid, tiles, 1, 0};
+  if (tiles <= grid) return s;
+  const int rounds = tiles / grid, rest = tiles - rounds * grid;
+  if (rest == 0) return s;
+  for (int f = max_f; f >= 2; f /= 2) {
+    if (f * rest <= grid) {
+      s.dp_tiles = rounds * grid;
+      s.tail_f = f;
+      s.tail_items = f * rest;
+      return s;
+    }
   }
   return s;
 }
 
 struct WorkItem {
-  int tile, kb0, kb1;
-  int sk_tile;  // -1: the whole tile is this CTA's; else index of the split tile
-  int slot;     // scratch slot of this CTA's partial (2c for its first run, 2c + 1 for its last)
+  int tile;   // 128 x BN tile index (M fastest)
+  int col0;   // first column of the item inside the tile
+  int width;  // columns of the item (BN, or BN / tail_f for a tail sub-tile)
 };
 
-// Walks one CTA's work items; every warp role walks the same sequence.  The
-// stream-K run comes first, so the fix-up of split tiles (reading the other
-// contributors' partials) overlaps the main loops of the whole tiles that follow.
+// Walks one CTA's work items; every warp role walks the same sequence.
 struct WorkWalker {
-  const SkSched& s;
-  int c, next_dp, u, u0, u1;
-  ZI_DEV WorkWalker(const SkSched& sched, int cta)
-      : s(sched), c(cta), next_dp(cta), u0(sched.base ? sched.unit_begin(cta) : 0),
-        u1(sched.base ? sched.unit_begin(cta + 1) : 0) {
-    u = u0;
-  }
+  const TailSched& s;
+  int c, next_dp;
+  bool tail_done;
+  ZI_DEV WorkWalker(const TailSched& sched, int cta) : s(sched), c(cta), next_dp(cta), tail_done(false) {}
+  template <int BN>
   ZI_DEV bool next(WorkItem& w) {
-    if (u < u1) {
-      const int st = u / s.kb, k0 = u % s.kb;
-      const int k1 = min(s.kb, k0 + (u1 - u));
-      w.tile = s.dp_tiles + st;
-      w.kb0 = k0;
-      w.kb1 = k1;
-      w.sk_tile = (k0 == 0 && k1 == s.kb) ? -1 : st;
-      w.slot = (u == u0) ? 2 * c : 2 * c + 1;
-      u += k1 - k0;
-      return true;
-    }
     if (next_dp < s.dp_tiles) {
       w.tile = next_dp;
-      w.kb0 = 0;
-      w.kb1 = s.kb;
-      w.sk_tile = -1;
-      w.slot = -1;
+      w.col0 = 0;
+      w.width = BN;
       next_dp += s.grid;
+      return true;
+    }
+    if (!tail_done && c < s.tail_items) {
+      tail_done = true;
+      w.width = BN / s.tail_f;
+      w.tile = s.dp_tiles + c / s.tail_f;
+      w.col0 = (c % s.tail_f) * w.width;
       return true;
     }
     return false;
   }
 };
 
-struct SplitScratch {
-  float* partials;  // [2 * G][128 * BN] fp32 (row-major, the accumulator tile as is)
-  int* counters;    // [max split tiles], zero on entry; reset to zero by each tile's finisher
-};
-
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                        int N, int K, EpiParams ep, SkSched sched, SplitScratch sk) {
+                        int N, int K, EpiParams ep, TailSched sched) {
   using L = GemmSmem<BN, STAGES>;
   constexpr int BM = 128, BK = 64;
   extern __shared__ uint8_t smem_raw[];
@@ -302,10 +277,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* ebar = drain + 1;  // syncs the 128 epilogue threads (bounded wait, unlike bar.sync)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
 
   if (device_error_set()) return;  // an earlier kernel timed out: leave everything untouched
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -320,7 +293,6 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
-    mbar_init(ebar, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -338,6 +310,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_m = (M + BM - 1) / BM;
+  const int KB = K / BK;
   WorkItem wi;
 
   if (warp == 0) {
@@ -345,18 +318,22 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       WorkWalker walk(sched, blockIdx.x);
-      while (ok && walk.next(wi)) {
-        const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
-        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
+      while (ok && walk.next<BN>(wi)) {
+        const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN + wi.col0;
+        const uint32_t bytes = L::kABytes + uint32_t(wi.width) * 128u;
+        for (int kb = 0; kb < KB; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + s * L::kStage;
-          mbar_arrive_expect_tx(&full[s], L::kStage);
+          mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
-          tma_load_2d(sa + L::kABytes, &tmB, &full[s], kb * BK, n0);
+          // B rows in 64-row boxes; consecutive boxes land 8 KB apart, which is the
+          // same swizzled layout one box of `width` rows would produce
+          for (int r64 = 0; r64 < wi.width / 64; ++r64)
+            tma_load_2d(sa + L::kABytes + r64 * 8192, &tmB, &full[s], kb * BK, n0 + r64 * 64);
           ++it;
         }
       }
@@ -372,12 +349,12 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
       uint32_t it = 0;
       int local = 0;
       bool ok = true;
       WorkWalker walk(sched, blockIdx.x);
-      while (ok && walk.next(wi)) {
+      while (ok && walk.next<BN>(wi)) {
+        const uint32_t idesc = idesc_bf16_f32(128, wi.width, false, false);
         const int acc = local & 1;
         const uint32_t u = uint32_t(local) >> 1;
         ++local;
@@ -387,7 +364,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * BN);
-        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
+        for (int kb = 0; kb < KB; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&full[s], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
             ok = false;
@@ -399,7 +376,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             tc_mma(d, smem_desc_sw128(a_addr + k * 32, 16), smem_desc_sw128(b_addr + k * 32, 16), idesc,
-                   (kb > wi.kb0 || k > 0) ? 1u : 0u);
+                   (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[s]);
           ++it;
@@ -417,79 +394,17 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;  // this warp's TMEM lane quarter
     const int row_in_tile = q * 32 + lane;
     int local = 0;
-    uint32_t ephase = 0;
-    auto epi_sync = [&]() -> bool {
-      mbar_arrive(ebar);
-      const bool r = mbar_wait(ebar, ephase, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE);
-      ephase ^= 1u;
-      return r;
-    };
     WorkWalker walk(sched, blockIdx.x);
-    while (walk.next(wi)) {
+    while (walk.next<BN>(wi)) {
       const int acc = local & 1;
       const uint32_t u = uint32_t(local) >> 1;
       ++local;
       if (!mbar_wait(&tfull[acc], u & 1u, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
+      const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN + wi.col0;
       const int row = m0 + row_in_tile;
       const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-      bool finish = true;
-      if (wi.sk_tile >= 0) {
-        // Split tile: publish this CTA's partial, and finish the tile only if last.
-        float* mine = sk.partials + size_t(wi.slot) * (128 * BN) + size_t(row_in_tile) * BN;
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32_sync(tb + c * 32, v);
-          float4* d4 = reinterpret_cast<float4*>(mine + c * 32);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            __stcg(d4 + k, make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
-        }
-        __threadfence();
-        if (!epi_sync()) break;
-        const int t0u = wi.sk_tile * sched.kb;
-        const int c_lo = sched.cta_of_unit(t0u), c_hi = sched.cta_of_unit(t0u + sched.kb - 1);
-        if (threadIdx.x == 64) {
-          const int old = atomicAdd(&sk.counters[wi.sk_tile], 1);
-          const bool last = old == c_hi - c_lo;
-          if (last) sk.counters[wi.sk_tile] = 0;  // ready for the next launch
-          *last_flag = last ? 1 : 0;
-        }
-        if (!epi_sync()) break;
-        finish = *last_flag != 0;
-        if (finish) {
-          __threadfence();
-          for (int c = 0; c < BN / 32; ++c) {
-            // The other contributor's partial for these 32 columns.  Every CTA's run is
-            // at least kb units long (the split part holds more than G tiles), so at
-            // most two runs meet in one tile: there is exactly one other partial.
-            int other = -1;
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              const int slot = sched.unit_begin(cc) >= t0u ? 2 * cc : 2 * cc + 1;
-              if (slot != wi.slot) other = slot;
-            }
-            float4 pa[8];
-            const float4* p4 = reinterpret_cast<const float4*>(sk.partials + size_t(other < 0 ? wi.slot : other) *
-                                                               (128 * BN) + size_t(row_in_tile) * BN + c * 32);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) pa[k] = other < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(p4 + k);
-            uint32_t v[32];
-            tmem_ld32_sync(tb + c * 32, v);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + pa[k].x);
-              v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + pa[k].y);
-              v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + pa[k].z);
-              v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + pa[k].w);
-            }
-            tmem_st32(tb + c * 32, v);
-          }
-          tmem_wait_st();
-        }
-      }
-      if (finish) gemm_epilogue<EPI, BN>(tb, row, row < M, n0, ep);
+      gemm_epilogue<EPI, BN>(tb, row, row < M, n0, wi.width, ep);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

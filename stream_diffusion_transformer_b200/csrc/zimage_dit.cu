@@ -156,43 +156,26 @@ enum KernelBit : unsigned {
 
 constexpr int kStages = 4;
 
-// Split scratch of the stream-K tail: 2 partial slots per persistent CTA (at
-// most kSkMaxGrid CTAs) of one 128 x 256 fp32 tile each, plus one counter per
-// split tile (fewer than 2 grids' worth).
-constexpr int kSkMaxGrid = 160;
-constexpr size_t kSkPartialBytes = size_t(2) * kSkMaxGrid * 128 * 256 * 4;
-constexpr size_t kSkCounterBytes = size_t(2) * kSkMaxGrid * 4;
-constexpr size_t kSkBytes = kSkPartialBytes + kSkCounterBytes;
-
-// `sk` (may be null) points at kSkBytes of scratch whose counters are zero.
 template <int BN, int EPI>
 int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint16_t* B, int M, int N, int K,
-             const EpiParams& ep, void* sk, cudaStream_t st) {
+             const EpiParams& ep, cudaStream_t st) {
   using L = GemmSmem<BN, kStages>;
-  static_assert(BN <= 256, "split slots hold 128 x 256 fp32");
   if (M <= 0) return ZI_OK;
   if (K % 64 != 0 || N % BN != 0 || K <= 0 || N <= 0) return ZI_ERR_SHAPE;
   CUtensorMap ta, tb;
   ZI_TRY(make_map(&ta, A, uint64_t(K), uint64_t(M), uint64_t(K) * 2, 64, 128));
-  ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, BN));
+  ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, 64));
   auto kern = gemm_bf16_tn_kernel<BN, kStages, EPI>;
   ZI_TRY(ensure_smem(dev, bit, kern, int(L::kBytes)));
   const int tiles = ((M + 127) / 128) * (N / BN);
-  int grid = tiles < dev->sms ? tiles : dev->sms;
-  if (sk && grid > kSkMaxGrid) grid = kSkMaxGrid;
-  const SkSched sched = make_sk_sched(tiles, grid, K / 64, sk != nullptr);
-  SplitScratch sp;
-  sp.partials = static_cast<float*>(sk);
-  sp.counters = sk ? reinterpret_cast<int*>(static_cast<uint8_t*>(sk) + kSkPartialBytes) : nullptr;
+  const int grid = tiles < dev->sms ? tiles : dev->sms;
+  // sub-tiles must stay 64-column multiples; a QKV sub-tile must hold whole
+  // 128-wide heads; SwiGLU pairs 128 gate with 128 up columns, so no split
+  const int max_f = (EPI == EPI_SWIGLU || EPI == EPI_UNPATCH) ? 1 : (EPI == EPI_QKV ? 2 : BN / 64);
+  const TailSched sched = make_tail_sched(tiles, grid, max_f < 4 ? max_f : 4);
   prof_pre(st);
-  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, N, K, ep, sched, sp);
+  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, N, K, ep, sched);
   return launched(kind, st);
-}
-
-int clear_split_counters(void* sk, cudaStream_t st) {
-  if (cudaMemsetAsync(static_cast<uint8_t*>(sk) + kSkPartialBytes, 0, kSkCounterBytes, st) != cudaSuccess)
-    return ZI_ERR_CUDA;
-  return ZI_OK;
 }
 
 EpiParams epi_plain(void* out, int ldo) {
@@ -254,7 +237,7 @@ constexpr size_t kAlign = 1024;
 inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-  size_t sk, mod, c, silu, hid, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
+  size_t mod, c, silu, hid, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
 };
 
 Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int mod_cols) {
@@ -265,7 +248,6 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   const size_t pairs = size_t(cfg.head_dim) / 2;
   Ws w;
   size_t o = 0;
-  w.sk = o; o = up(o + kSkBytes);
   w.mod = o; o = up(o + size_t(batch) * size_t(mod_cols) * 4);
   w.c = o; o = up(o + (model ? size_t(batch) * 256 * 4 : 0));
   w.silu = o; o = up(o + (model ? size_t(batch) * 256 * 4 : 0));
@@ -341,7 +323,6 @@ struct BlockCtx {
   const float2* rope;
   const float* mod;  // this block's 4D modulation inside the per-batch vector, or null
   int mod_ld;
-  void* sk;          // stream-K split scratch (counters zero)
   int nseg;
   int seg_row0[2], seg_len[2];  // local rows
 };
@@ -359,9 +340,9 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   eq.dim = D;
   eq.row_off = b.row_off;
   eq.map = b.map;
-  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, b.sk, st)));
+  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st)));
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len, st));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D, epi_plain(b.o, D), b.sk, st)));
+  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D, epi_plain(b.o, D), st)));
   PostParams pa;
   memset(&pa, 0, sizeof(pa));
   pa.x_in = b.x_in;
@@ -383,8 +364,8 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   pa.eps_ln = b.cfg->final_eps;
   ZI_TRY(run_post(pa, b.rows, st));
   ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp, D, epi_plain(b.u, Fp),
-                                    b.sk, st)));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp, epi_plain(b.o, D), b.sk, st)));
+                                    st)));
+  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp, epi_plain(b.o, D), st)));
   PostParams pf = pa;
   pf.x_in = b.x_out;
   pf.g_post = b.w->g_ffn2;
@@ -572,25 +553,14 @@ int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, float* d_co
   return run_rope(*cfg, d_pos, n, reinterpret_cast<float2*>(d_cos_sin), reinterpret_cast<cudaStream_t>(stream));
 }
 
-int zi_gemm_workspace_size(size_t* h_bytes) {
-  if (!h_bytes) return ZI_ERR_ARG;
-  *h_bytes = kSkBytes;
-  return ZI_OK;
-}
-
-int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, void* d_ws,
-                 size_t ws_bytes, zi_stream_t stream) {
+int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, zi_stream_t stream) {
   if (!d_a || !d_b || !d_c || m < 0 || n <= 0 || k <= 0) return ZI_ERR_ARG;
   if (!aligned16(d_a) || !aligned16(d_b) || !aligned16(d_c)) return ZI_ERR_ALIGN;
   if (k % 64 || n % 256) return ZI_ERR_SHAPE;
-  if (d_ws && (ws_bytes < kSkBytes)) return ZI_ERR_WORKSPACE;
-  if (d_ws && (reinterpret_cast<uintptr_t>(d_ws) & 255u)) return ZI_ERR_ALIGN;
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d_ws) ZI_TRY(clear_split_counters(d_ws, st));
-  return run_gemm<256, EPI_BF16>(dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM, d_a, d_b, m, n, k, epi_plain(d_c, n), d_ws,
-                                 st);
+  return run_gemm<256, EPI_BF16>(dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM, d_a, d_b, m, n, k, epi_plain(d_c, n),
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads, zi_stream_t stream) {
@@ -657,8 +627,6 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.rope = rope;
   b.mod = modulated ? mod : nullptr;
   b.mod_ld = 4 * D;
-  b.sk = ws + L.sk;
-  ZI_TRY(clear_split_counters(b.sk, st));
   b.nseg = 1;
   b.seg_row0[0] = 0;
   b.seg_len[0] = seq;
@@ -738,7 +706,6 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
   uint16_t* capn = reinterpret_cast<uint16_t*>(ws + L.capn);
   const RowMap map{rows_img, s_img, s_txt};
   const float eps = cfg->norm_eps;
-  ZI_TRY(clear_split_counters(ws + L.sk, st));
 
   // timestep conditioning and every adaLN projection
   {
@@ -792,12 +759,12 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
     ZI_TRY(launched(ZI_KERNEL_PATCHIFY, st));
     EpiParams ex = epi_plain(x, D);
     ex.bias = w->x_emb_b;
-    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, tok, w->x_emb_w, rows_img, D, 64, ex, ws + L.sk, st)));
+    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, tok, w->x_emb_w, rows_img, D, 64, ex, st)));
     ZI_TRY(run_rms_mod<uint16_t>(d_txt, rows_txt, cfg->cap_dim, w->cap_norm, nullptr, 0, map, rows_img, eps, capn,
                                  st));
     EpiParams ec = epi_plain(x + size_t(rows_img) * D, D);
     ec.bias = w->cap_b;
-    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, capn, w->cap_w, rows_txt, D, cfg->cap_dim, ec, ws + L.sk, st)));
+    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, capn, w->cap_w, rows_txt, D, cfg->cap_dim, ec, st)));
   }
 
   BlockCtx base;
@@ -807,7 +774,6 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
   base.map = map;
   base.rope = rope;
   base.mod_ld = mod_ld;
-  base.sk = ws + L.sk;
 
   auto segment_ctx = [&](int row_off, int nrows, int seglen) {
     BlockCtx b = base;
@@ -891,7 +857,7 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
     ef.lat_c = cfg->in_ch;
     ef.lat_h = lat_h;
     ef.lat_w = lat_w;
-    ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, ZI_KERNEL_GEMM_FINAL, h, w->final_w, rows_img, 4 * cfg->in_ch, D, ef, nullptr, st)));
+    ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, ZI_KERNEL_GEMM_FINAL, h, w->final_w, rows_img, 4 * cfg->in_ch, D, ef, st)));
   }
   return ZI_OK;
 }

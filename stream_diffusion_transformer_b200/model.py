@@ -184,18 +184,13 @@ def rope_table(cfg: abi.ZiConfig, pos: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def gemm(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None, split: bool = True) -> torch.Tensor:
-    """a bf16 [M, K] @ b bf16 [N, K]^T -> bf16 [M, N]; split=True gives the kernel split scratch."""
+def gemm(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """a bf16 [M, K] @ b bf16 [N, K]^T -> bf16 [M, N]."""
     M, K = a.shape
     N = b.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
-    ws = None
-    if split:
-        n = ctypes.c_size_t(0)
-        abi.call("zi_gemm_workspace_size", ctypes.byref(n))
-        ws = torch.empty(n.value, dtype=torch.uint8, device=a.device)
-    abi.call("zi_gemm_bf16", _p(a), _p(b), _p(out), M, N, K, _p(ws), 0 if ws is None else ws.numel(), _stream())
+    abi.call("zi_gemm_bf16", _p(a), _p(b), _p(out), M, N, K, _stream())
     return out
 
 
