@@ -266,8 +266,9 @@ struct WorkWalker {
 
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
-    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                        int N, int K, EpiParams ep, TailSched sched) {
+    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB64, int M, int N, int K, EpiParams ep,
+                        TailSched sched) {
   using L = GemmSmem<BN, STAGES>;
   constexpr int BM = 128, BK = 64;
   extern __shared__ uint8_t smem_raw[];
@@ -299,6 +300,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
@@ -330,10 +332,14 @@ __global__ void __launch_bounds__(192, 1)
           uint8_t* sa = smem + s * L::kStage;
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
-          // B rows in 64-row boxes; consecutive boxes land 8 KB apart, which is the
-          // same swizzled layout one box of `width` rows would produce
-          for (int r64 = 0; r64 < wi.width / 64; ++r64)
-            tma_load_2d(sa + L::kABytes + r64 * 8192, &tmB, &full[s], kb * BK, n0 + r64 * 64);
+          if (wi.width == BN) {
+            tma_load_2d(sa + L::kABytes, &tmB, &full[s], kb * BK, n0);
+          } else {
+            // a tail sub-tile: its B rows in 64-row boxes, which land 8 KB apart in
+            // the same swizzled layout one box of `width` rows would produce
+            for (int r64 = 0; r64 < wi.width / 64; ++r64)
+              tma_load_2d(sa + L::kABytes + r64 * 8192, &tmB64, &full[s], kb * BK, n0 + r64 * 64);
+          }
           ++it;
         }
       }

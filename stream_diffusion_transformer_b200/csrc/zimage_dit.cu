@@ -162,9 +162,10 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint
   using L = GemmSmem<BN, kStages>;
   if (M <= 0) return ZI_OK;
   if (K % 64 != 0 || N % BN != 0 || K <= 0 || N <= 0) return ZI_ERR_SHAPE;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tb64;
   ZI_TRY(make_map(&ta, A, uint64_t(K), uint64_t(M), uint64_t(K) * 2, 64, 128));
-  ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, 64));
+  ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, BN));
+  ZI_TRY(make_map(&tb64, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, 64));
   auto kern = gemm_bf16_tn_kernel<BN, kStages, EPI>;
   ZI_TRY(ensure_smem(dev, bit, kern, int(L::kBytes)));
   const int tiles = ((M + 127) / 128) * (N / BN);
@@ -174,7 +175,7 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint
   const int max_f = (EPI == EPI_SWIGLU || EPI == EPI_UNPATCH) ? 1 : (EPI == EPI_QKV ? 2 : BN / 64);
   const TailSched sched = make_tail_sched(tiles, grid, max_f < 4 ? max_f : 4);
   prof_pre(st);
-  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, N, K, ep, sched);
+  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, tb64, M, N, K, ep, sched);
   return launched(kind, st);
 }
 
