@@ -69,24 +69,26 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
+    """Hash of the CUDA sources a kernel is built from (names under the package's csrc/)."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "stream_diffusion_transformer_b200", "csrc")
-    for name in sorted(os.listdir(cdir)):
+    for name in sorted(files):
         with open(os.path.join(cdir, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json), or None
+    if there is none or the kernel's sources changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
         rec = json.load(fh)
     e = rec.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("sources", [])):
         return None
     return e.get("dram_bytes_per_launch")
 
