@@ -1,20 +1,20 @@
 // Non-causal flash attention (head_dim 128, bf16 in/out, fp32 softmax) on tcgen05.
 //
-// One CTA per (128-query tile, head, batch element), 6 warps:
-//   warp 0      TMA: Q tile once, then K and V tiles (128 keys each) into
+// One CTA per (pair of 128-query tiles A and B, head, batch element), 10 warps:
+//   warp 0      TMA: both Q tiles once, then K and V tiles (128 keys each) into
 //               2-deep rings, straight out of the fused [rows, 3D] projection
 //               buffer (the head's 128 columns as two 64-wide swizzled boxes)
-//   warp 1      TMEM allocator + tcgen05.mma issuer:
-//                 S_j = Q K_j^T          (A = Q smem, B = K smem, both K-major)
-//                 O  += P_{j-1} V_{j-1}  (A = P smem K-major, B = V smem MN-major)
-//               S is double-buffered in TMEM (2 x 128 columns), O lives in TMEM
-//               (128 columns); S_{j+1} is issued before P_j V_j so the tensor
-//               core keeps working while the softmax warps exponentiate.
-//   warps 2..5  softmax: one thread per query row (its TMEM lane), online
-//               softmax in the exp2 domain with a lazily updated running max
-//               (O in TMEM is rescaled only when a row's max grows by more
-//               than 2^8), P written to smem as bf16 in the swizzled layout
-//               the MMA reads; final O / l written as bf16.
+//   warp 1      TMEM allocator + tcgen05.mma issuer.  TMEM: S_A, S_B, O_A, O_B,
+//               128 columns each.  Per key tile j the tensor core runs
+//                 S_A(j+1) = Q_A K^T, O_B += P_B(j) V, S_B(j+1) = Q_B K^T, O_A += P_A(j+1) V
+//               so each tile's softmax has the other tile's two MMAs to hide behind.
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: one thread per
+//               query row (its TMEM lane); online softmax in the exp2 domain with a
+//               lazily updated running max (O rescaled in TMEM only when a row's max
+//               grows by more than 2^8); P (bf16) is written back over the first 64
+//               columns of its S and read from TMEM by the PV MMA.
+// A tcgen05.mma that overwrites S(j+1) is issued after the MMA that reads P(j)
+// from the same columns; the tensor core executes one CTA's MMAs in issue order.
 // The key sequence of a batch element can be split over two row segments of
 // the token buffer (image rows and text rows); key tiles that run past a
 // segment's end are masked to -inf.
@@ -30,15 +30,18 @@ struct AttnParams {
   int nseg;       // 1 or 2
   int seg_row0[2];  // first row of segment i for batch element 0
   int seg_len[2];   // rows per batch element in segment i (element b starts at row0 + b * len)
+  int q_tiles;      // query tiles per batch element (both segments)
   float scale_log2; // log2(e) / sqrt(head_dim)
 };
 
 namespace attn {
+constexpr int kThreads = 320;
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile (two 64-column halves)
 constexpr uint32_t kHalf = kTile / 2;
-constexpr uint32_t kQ = 0, kK0 = kTile, kV0 = 3 * kTile, kP = 5 * kTile;
+constexpr uint32_t kQ0 = 0, kK0 = 2 * kTile, kV0 = 4 * kTile;
 constexpr uint32_t kBar = 6 * kTile;
 constexpr uint32_t kSmemBytes = kBar + 256 + 1024;
+constexpr uint32_t kColS = 0, kColO = 256;  // S_t at kColS + 128 t, O_t at kColO + 128 t
 }  // namespace attn
 
 ZI_DEV void attn_tile_rows(const AttnParams& p, int b, int tile, int& row0, int& valid) {
@@ -53,7 +56,46 @@ ZI_DEV void attn_tile_rows(const AttnParams& p, int b, int tile, int& row0, int&
   valid = min(128, p.seg_len[seg] - t * 128);
 }
 
-__global__ void __launch_bounds__(192, 1)
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, A (bf16) read from TMEM.
+ZI_DEV void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+ZI_DEV float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pair arithmetic (one instruction for two values).
+ZI_DEV uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+ZI_DEV void f2_unpack(uint64_t v, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
+ZI_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+ZI_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+ZI_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__global__ void __launch_bounds__(attn::kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm, AttnParams p) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
@@ -64,13 +106,11 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* k_empty = bars + 3;  // [2]
   uint64_t* v_full = bars + 5;   // [2]
   uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* s_free = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* p_free = bars + 14;
-  uint64_t* o_full = bars + 15;
-  uint64_t* drain = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* s_full = bars + 9;   // [2 tiles]
+  uint64_t* p_full = bars + 11;  // [2 tiles]
+  uint64_t* pv_done = bars + 13; // [2 tiles]
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (device_error_set()) return;
@@ -78,6 +118,8 @@ __global__ void __launch_bounds__(192, 1)
   const int head = blockIdx.y, b = blockIdx.z;
   int n_kv = (p.seg_len[0] + 127) / 128;
   if (p.nseg > 1) n_kv += (p.seg_len[1] + 127) / 128;
+  const int tile_a = 2 * blockIdx.x;
+  const bool has_b = tile_a + 1 < p.q_tiles;  // CTA-uniform: the last CTA may hold one tile
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -87,11 +129,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(p_free, 1);
-    mbar_init(o_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -105,16 +145,20 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  int q_row0, q_valid;
-  attn_tile_rows(p, b, blockIdx.x, q_row0, q_valid);
   const int colq = head * 128, colk = p.dim + head * 128, colv = 2 * p.dim + head * 128;
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kTile);
-      tma_load_2d(smem + kQ, &tm, q_full, colq, q_row0);
-      tma_load_2d(smem + kQ + kHalf, &tm, q_full, colq + 64, q_row0);
+      int qa0, qav, qb0 = 0, qbv = 0;
+      attn_tile_rows(p, b, tile_a, qa0, qav);
+      if (has_b) attn_tile_rows(p, b, tile_a + 1, qb0, qbv);
+      mbar_arrive_expect_tx(q_full, has_b ? 2 * kTile : kTile);
+      tma_load_2d(smem + kQ0, &tm, q_full, colq, qa0);
+      tma_load_2d(smem + kQ0 + kHalf, &tm, q_full, colq + 64, qa0);
+      if (has_b) {
+        tma_load_2d(smem + kQ0 + kTile, &tm, q_full, colq, qb0);
+        tma_load_2d(smem + kQ0 + kTile + kHalf, &tm, q_full, colq + 64, qb0);
+      }
       uint32_t issued_k = 0, issued_v = 0;
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
@@ -146,164 +190,190 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
-      const uint32_t q_addr = smem_u32(smem + kQ);
-      const uint32_t p_addr = smem_u32(smem + kP);
+      const int ntile = has_b ? 2 : 1;
       bool ok = mbar_wait(q_full, 0, abort_flag, ZI_DEVERR_TIMEOUT_MMA);
       tc_fence_after();
-      auto issue_pv = [&](int jj) -> bool {
-        const int bb = jj & 1;
-        const uint32_t rr = uint32_t(jj) >> 1;
-        if (!mbar_wait(p_full, uint32_t(jj) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) return false;
-        if (!mbar_wait(&v_full[bb], rr & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + kV0 + bb * kTile);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t ad = smem_desc_sw128(p_addr + (k >> 2) * kHalf + (k & 3) * 32, 16);
-          const uint64_t bd = smem_desc_sw128(v_addr + k * 2048, kHalf);
-          tc_mma(tmem + 256, ad, bd, idesc_o, (jj > 0 || k > 0) ? 1u : 0u);
-        }
-        tc_commit(&v_empty[bb]);
-        tc_commit(p_free);
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int bi = j & 1;
-        const uint32_t r = uint32_t(j) >> 1;
-        if (!mbar_wait(&k_full[bi], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) { ok = false; break; }
-        if (!mbar_wait(&s_free[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + kK0 + bi * kTile);
+      // S_t(j) = Q_t K_j^T into S_t
+      auto issue_s = [&](int t, int j) {
+        const uint32_t q_addr = smem_u32(smem + kQ0 + t * kTile);
+        const uint32_t k_addr = smem_u32(smem + kK0 + (j & 1) * kTile);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint64_t ad = smem_desc_sw128(q_addr + (k >> 2) * kHalf + (k & 3) * 32, 16);
           const uint64_t bd = smem_desc_sw128(k_addr + (k >> 2) * kHalf + (k & 3) * 32, 16);
-          tc_mma(tmem + uint32_t(bi * 128), ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          tc_mma(tmem + kColS + 128 * t, ad, bd, idesc_s, k > 0 ? 1u : 0u);
         }
-        tc_commit(&k_empty[bi]);
-        tc_commit(&s_full[bi]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
-      }
-      if (ok && issue_pv(n_kv - 1)) {
-        tc_commit(o_full);
+        tc_commit(&s_full[t]);
+      };
+      // O_t += P_t(j) V_j, P_t (bf16, 64 columns) read from the front of S_t
+      auto issue_pv = [&](int t, int j) -> bool {
+        if (!mbar_wait(&p_full[t], uint32_t(j) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + kV0 + (j & 1) * kTile);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t bd = smem_desc_sw128(v_addr + k * 2048, kHalf);
+          tc_mma_ts(tmem + kColO + 128 * t, tmem + kColS + 128 * t + 8 * k, bd, idesc_o,
+                    (j > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(&pv_done[t]);
+        return true;
+      };
+      auto wait_k = [&](int j) {
+        return mbar_wait(&k_full[j & 1], (uint32_t(j) >> 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA);
+      };
+      auto wait_v = [&](int j) {
+        return mbar_wait(&v_full[j & 1], (uint32_t(j) >> 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA);
+      };
+      // prologue: S_A(0), S_B(0), O_A += P_A(0) V_0
+      if (ok && wait_k(0)) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (ntile > 1) issue_s(1, 0);
+        tc_commit(&k_empty[0]);
+        ok = wait_v(0) && issue_pv(0, 0);
       } else {
+        ok = false;
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const bool more = j + 1 < n_kv;
+        if (more) {
+          if (!wait_k(j + 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (ntile > 1 && !issue_pv(1, j)) { ok = false; break; }
+        tc_commit(&v_empty[j & 1]);
+        if (more) {
+          if (ntile > 1) issue_s(1, j + 1);
+          tc_commit(&k_empty[(j + 1) & 1]);
+          if (!wait_v(j + 1) || !issue_pv(0, j + 1)) { ok = false; break; }
+        }
+      }
+      if (!ok) {
         tc_commit(drain);
         volatile int never = 0;
         mbar_wait(drain, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
       }
     }
   } else {
+    // softmax warpgroups: t = 0 (warps 2..5) handles tile A, t = 1 (warps 6..9) tile B
+    const int t = (warp - 2) >> 2;
     const int q = warp & 3;
     const int i = q * 32 + lane;  // query row in the tile == TMEM lane
-    const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
-    const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l = 0.f;
-    uint32_t s[128];
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int bi = j & 1;
-      const uint32_t r = uint32_t(j) >> 1;
-      int kv0, kvn;
-      attn_tile_rows(p, b, j, kv0, kvn);
-      if (!mbar_wait(&s_full[bi], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(lane_addr + uint32_t(bi * 128 + c * 32), &s[c * 32]);
-      }
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence32(&s[c * 32]);
-      tc_fence_before();
-      mbar_arrive(&s_free[bi]);
-
-      // Row max and row sum use 8 independent chains each, so the per-element
-      // FMNMX / FFMA / EX2 / FADD of different columns overlap instead of
-      // waiting on one serial dependency chain.
-      if (kvn < 128) {  // the segment's last key tile: mask the columns past its end
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= kvn) s[c] = __float_as_uint(-INFINITY);
-      }
-      float mxs[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mxs[k] = __uint_as_float(s[k]);
-#pragma unroll
-      for (int c = 8; c < 128; ++c) mxs[c & 7] = fmaxf(mxs[c & 7], __uint_as_float(s[c]));
-      const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                             fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const bool need = m_new > m_run + 8.0f;
-      float alpha = 1.0f;
-      const bool resc = __any_sync(0xffffffffu, need);
-      if (resc) {
-        alpha = fast_exp2(m_run - m_new);
-        m_run = m_new;
-        l *= alpha;
-      }
-      const float neg_m = -m_run;
-      float sums[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sums[k] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float e = fast_exp2(fmaf(__uint_as_float(s[c]), sl2, neg_m));
-        sums[c & 7] += e;
-        s[c] = __float_as_uint(e);
-      }
-      l += ((sums[0] + sums[1]) + (sums[2] + sums[3])) + ((sums[4] + sums[5]) + (sums[6] + sums[7]));
-      if (j >= 1) {
-        if (!mbar_wait(p_free, uint32_t(j - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) { ok = false; break; }
+    if (t == 0 || has_b) {
+      int q_row0, q_valid;
+      attn_tile_rows(p, b, tile_a + t, q_row0, q_valid);
+      const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
+      const uint32_t s_addr = lane_addr + kColS + 128 * t;
+      const uint32_t o_addr = lane_addr + kColO + 128 * t;
+      const float sl2 = p.scale_log2;
+      float m_run = -INFINITY, l = 0.f;
+      uint32_t s[128];
+      bool ok = true;
+      for (int j = 0; j < n_kv; ++j) {
+        int kv0, kvn;
+        attn_tile_rows(p, b, j, kv0, kvn);
+        if (!mbar_wait(&s_full[t], uint32_t(j) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) { ok = false; break; }
         tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, &s[c * 32]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence32(&s[c * 32]);
+        if (kvn < 128) {  // the segment's last key tile: mask the columns past its end
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= kvn) s[c] = __float_as_uint(-INFINITY);
+        }
+        // row max: 3-input max over 8 independent chains
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(s[k]);
+#pragma unroll
+        for (int c = 8; c < 120; c += 16) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = max3f(mx8[k], __uint_as_float(s[c + k]), __uint_as_float(s[c + 8 + k]));
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s[120 + k]));
+        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const bool resc = __any_sync(0xffffffffu, m_new > m_run + 8.0f);
+        float alpha = 1.0f;
         if (resc) {
+          alpha = fast_exp2(m_run - m_new);
+          m_run = m_new;
+          l *= alpha;
+        }
+        // p = 2^(s * sl2 - m): packed FMA, MUFU exp2, packed row sums, bf16 pairs
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm = f2_pack(-m_run, -m_run);
+        uint64_t sum2[4] = {0, 0, 0, 0};
+        uint32_t pw[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2x2, negm), x0, x1);
+          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(e0, e1));
+          pw[c] = pack_bf16x2(e0, e1);
+        }
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2_unpack(sum2[0], a0, a1);
+          f2_unpack(sum2[1], b0, b1);
+          f2_unpack(sum2[2], c0, c1);
+          f2_unpack(sum2[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
+        if (resc && j > 0) {
+          // O_t holds PV up to tile j-1: wait for that MMA, then scale O_t by alpha
+          if (!mbar_wait(&pv_done[t], uint32_t(j - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32_sync(lane_addr + 256 + c * 32, o);
+            tmem_ld32_sync(o_addr + c * 32, o);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(lane_addr + 256 + c * 32, o);
+            for (int k = 0; k < 16; ++k) {
+              float y0, y1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1])), a2), y0, y1);
+              o[2 * k] = __float_as_uint(y0);
+              o[2 * k + 1] = __float_as_uint(y1);
+            }
+            tmem_st32(o_addr + c * 32, o);
           }
-          tmem_wait_st();
         }
+        // P over the first 64 columns of S_t (S_t(j) is already in registers)
+        tmem_st32(s_addr, &pw[0]);
+        tmem_st32(s_addr + 32, &pw[32]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
       }
-      // P row i -> smem, two 64-column halves, 16-byte chunks swizzled by (i & 7)
-      uint8_t* prow = smem + kP + i * 128;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const int c0 = h * 64 + c8 * 8;
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(s[c0 + 0]), __uint_as_float(s[c0 + 1]));
-          w.y = pack_bf16x2(__uint_as_float(s[c0 + 2]), __uint_as_float(s[c0 + 3]));
-          w.z = pack_bf16x2(__uint_as_float(s[c0 + 4]), __uint_as_float(s[c0 + 5]));
-          w.w = pack_bf16x2(__uint_as_float(s[c0 + 6]), __uint_as_float(s[c0 + 7]));
-          *reinterpret_cast<uint4*>(prow + h * kHalf + ((c8 ^ (i & 7)) << 4)) = w;
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    if (ok && mbar_wait(o_full, 0, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) {
-      tc_fence_after();
-      const float inv = 1.0f / l;
-      uint16_t* orow = p.out + size_t(q_row0 + i) * p.ldo + head * 128;
+      if (ok && mbar_wait(&pv_done[t], uint32_t(n_kv - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) {
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        uint16_t* orow = p.out + size_t(q_row0 + i) * p.ldo + head * 128;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32_sync(lane_addr + 256 + c * 32, o);
-        if (i < q_valid) {
-          uint4* d = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32_sync(o_addr + c * 32, o);
+          if (i < q_valid) {
+            uint4* d = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-            d[k] = w;
+            for (int k = 0; k < 4; ++k) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+              d[k] = w;
+            }
           }
         }
       }

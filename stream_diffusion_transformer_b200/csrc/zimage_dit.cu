@@ -208,9 +208,10 @@ int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out
     if (i < nseg) qt += (len[i] + 127) / 128;
   }
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(128.0));
-  dim3 grid(qt, heads, batch);
+  p.q_tiles = qt;
+  dim3 grid((qt + 1) / 2, heads, batch);  // two query tiles per CTA
   prof_pre(st);
-  attention_kernel<<<grid, 192, attn::kSmemBytes, st>>>(tm, p);
+  attention_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(tm, p);
   return launched(ZI_KERNEL_ATTENTION, st);
 }
 
