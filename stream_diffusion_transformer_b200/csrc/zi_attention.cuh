@@ -1,14 +1,17 @@
 // Non-causal flash attention (head_dim 128, bf16 in/out, fp32 softmax) on tcgen05.
 //
-// One CTA per (pair of 128-query tiles A and B, head, batch element), 10 warps:
-//   warp 0      TMA: both Q tiles once, then K and V tiles (128 keys each) into
+// One CTA per (pair of 128-query tiles A and B, head, batch element), 12 warps
+// in three warpgroups; registers move from the third to the first two with
+// setmaxnreg (launch 168 per thread; softmax 216, TMA/MMA 56):
+//   warp 8      TMA: both Q tiles once, then K and V tiles (128 keys each) into
 //               2-deep rings, straight out of the fused [rows, 3D] projection
 //               buffer (the head's 128 columns as two 64-wide swizzled boxes)
-//   warp 1      TMEM allocator + tcgen05.mma issuer.  TMEM: S_A, S_B, O_A, O_B,
+//   warp 9      TMEM allocator + tcgen05.mma issuer.  TMEM: S_A, S_B, O_A, O_B,
 //               128 columns each.  Per key tile j the tensor core runs
 //                 S_A(j+1) = Q_A K^T, O_B += P_B(j) V, S_B(j+1) = Q_B K^T, O_A += P_A(j+1) V
 //               so each tile's softmax has the other tile's two MMAs to hide behind.
-//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: one thread per
+//   warps 10-11 idle
+//   warps 0..3  softmax of tile A, warps 4..7 softmax of tile B: one thread per
 //               query row (its TMEM lane); online softmax in the exp2 domain with a
 //               lazily updated running max (O rescaled in TMEM only when a row's max
 //               grows by more than 2^8); P (bf16) is written back over the first 64
@@ -35,7 +38,9 @@ struct AttnParams {
 };
 
 namespace attn {
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kRegsSoftmax = 216;  // 2 x 128 x 216 + 128 x 56 = 62464 <= 384 x 168 registers at launch
+constexpr int kRegsOther = 56;
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile (two 64-column halves)
 constexpr uint32_t kHalf = kTile / 2;
 constexpr uint32_t kQ0 = 0, kK0 = 2 * kTile, kV0 = 4 * kTile;
@@ -136,8 +141,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tm);
-  if (warp == 1) {
+  if (warp == 8 && lane == 0) prefetch_tmap(&tm);
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -147,7 +152,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int colq = head * 128, colk = p.dim + head * 128, colv = 2 * p.dim + head * 128;
 
-  if (warp == 0) {
+  // Each role's code sits inside the branch that set its register budget, so the
+  // register allocator sees the budget that holds for it.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+   if (warp == 8) {
     if (lane == 0) {
       int qa0, qav, qb0 = 0, qbv = 0;
       attn_tile_rows(p, b, tile_a, qa0, qav);
@@ -186,7 +195,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           mbar_wait(&v_full[j & 1], (j >> 1) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
@@ -256,9 +265,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         mbar_wait(drain, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
       }
     }
+   }
   } else {
-    // softmax warpgroups: t = 0 (warps 2..5) handles tile A, t = 1 (warps 6..9) tile B
-    const int t = (warp - 2) >> 2;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    // softmax warpgroups: t = 0 (warps 0..3) handles tile A, t = 1 (warps 4..7) tile B
+    const int t = warp >> 2;
     const int q = warp & 3;
     const int i = q * 32 + lane;  // query row in the tile == TMEM lane
     if (t == 0 || has_b) {
@@ -381,7 +392,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
