@@ -3,14 +3,15 @@
 // One CTA per (pair of 128-query tiles A and B, head, batch element), 12 warps
 // in three warpgroups; registers move from the third to the first two with
 // setmaxnreg (launch 168 per thread; softmax 216, TMA/MMA 56):
-//   warp 8      TMA: both Q tiles once, then K and V tiles (128 keys each) into
-//               2-deep rings, straight out of the fused [rows, 3D] projection
+//   warp 8      TMA: both Q tiles once, then K tiles (128 keys each) into a
+//               2-deep ring, straight out of the fused [rows, 3D] projection
 //               buffer (the head's 128 columns as two 64-wide swizzled boxes)
 //   warp 9      TMEM allocator + tcgen05.mma issuer.  TMEM: S_A, S_B, O_A, O_B,
 //               128 columns each.  Per key tile j the tensor core runs
 //                 S_A(j+1) = Q_A K^T, O_B += P_B(j) V, S_B(j+1) = Q_B K^T, O_A += P_A(j+1) V
 //               so each tile's softmax has the other tile's two MMAs to hide behind.
-//   warps 10-11 idle
+//   warp 10     TMA for the V ring (warp 8 then only loads Q and K)
+//   warp 11     idle
 //   warps 0..3  softmax of tile A, warps 4..7 softmax of tile B: one thread per
 //               query row (its TMEM lane); online softmax in the exp2 domain with a
 //               lazily updated running max (O rescaled in TMEM only when a row's max
@@ -100,6 +101,29 @@ ZI_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x for a pair on the FMA pipe (FlashAttention-4's relief for the 16/clk/SM
+// MUFU): Cody-Waite split x = n + f with n = rint(x) (the 1.5 * 2^23 rounding
+// trick), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients were
+// fitted here by the Remez exchange algorithm on the relative error (max
+// relative error 7.5e-5, far below the bf16 rounding P gets next); n is added
+// to the exponent field.  x is clamped at -126 so the result stays normal.
+ZI_DEV void exp2_poly_pair(float x0, float x1, float& e0, float& e1) {
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  const uint64_t x2 = f2_pack(x0, x1);
+  const uint64_t t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t n2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t fr = f2_fma(n2, f2_pack(-1.0f, -1.0f), x2);
+  uint64_t p2 = f2_fma(f2_pack(0.05517166853f, 0.05517166853f), fr, f2_pack(0.2426111251f, 0.2426111251f));
+  p2 = f2_fma(p2, fr, f2_pack(0.6932609677f, 0.6932609677f));
+  p2 = f2_fma(p2, fr, f2_pack(0.9999280572f, 0.9999280572f));
+  float t0, t1, p0, p1;
+  f2_unpack(t2, t0, t1);
+  f2_unpack(p2, p0, p1);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __global__ void __launch_bounds__(attn::kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm, AttnParams p) {
   using namespace attn;
@@ -156,43 +180,45 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   // register allocator sees the budget that holds for it.
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-   if (warp == 8) {
+   if (warp == 8 || warp == 10) {
+    // warp 8 loads Q and the K ring, warp 10 the V ring, so neither ring's wait
+    // holds up the other's next load
     if (lane == 0) {
-      int qa0, qav, qb0 = 0, qbv = 0;
-      attn_tile_rows(p, b, tile_a, qa0, qav);
-      if (has_b) attn_tile_rows(p, b, tile_a + 1, qb0, qbv);
-      mbar_arrive_expect_tx(q_full, has_b ? 2 * kTile : kTile);
-      tma_load_2d(smem + kQ0, &tm, q_full, colq, qa0);
-      tma_load_2d(smem + kQ0 + kHalf, &tm, q_full, colq + 64, qa0);
-      if (has_b) {
-        tma_load_2d(smem + kQ0 + kTile, &tm, q_full, colq, qb0);
-        tma_load_2d(smem + kQ0 + kTile + kHalf, &tm, q_full, colq + 64, qb0);
+      const bool kq = warp == 8;
+      if (kq) {
+        int qa0, qav, qb0 = 0, qbv = 0;
+        attn_tile_rows(p, b, tile_a, qa0, qav);
+        if (has_b) attn_tile_rows(p, b, tile_a + 1, qb0, qbv);
+        mbar_arrive_expect_tx(q_full, has_b ? 2 * kTile : kTile);
+        tma_load_2d(smem + kQ0, &tm, q_full, colq, qa0);
+        tma_load_2d(smem + kQ0 + kHalf, &tm, q_full, colq + 64, qa0);
+        if (has_b) {
+          tma_load_2d(smem + kQ0 + kTile, &tm, q_full, colq, qb0);
+          tma_load_2d(smem + kQ0 + kTile + kHalf, &tm, q_full, colq + 64, qb0);
+        }
       }
-      uint32_t issued_k = 0, issued_v = 0;
+      uint64_t* fullb = kq ? k_full : v_full;
+      uint64_t* emptyb = kq ? k_empty : v_empty;
+      const uint32_t base = kq ? kK0 : kV0;
+      const int col = kq ? colk : colv;
+      uint32_t issued = 0;
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
+      for (int j = 0; j < n_kv; ++j) {
         const int bi = j & 1;
         const uint32_t r = uint32_t(j) >> 1;
         int kv0, kvn;
         attn_tile_rows(p, b, j, kv0, kvn);
-        if (!mbar_wait(&k_empty[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) { ok = false; break; }
-        mbar_arrive_expect_tx(&k_full[bi], kTile);
-        tma_load_2d(smem + kK0 + bi * kTile, &tm, &k_full[bi], colk, kv0);
-        tma_load_2d(smem + kK0 + bi * kTile + kHalf, &tm, &k_full[bi], colk + 64, kv0);
-        ++issued_k;
-        if (!mbar_wait(&v_empty[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) { ok = false; break; }
-        mbar_arrive_expect_tx(&v_full[bi], kTile);
-        tma_load_2d(smem + kV0 + bi * kTile, &tm, &v_full[bi], colv, kv0);
-        tma_load_2d(smem + kV0 + bi * kTile + kHalf, &tm, &v_full[bi], colv + 64, kv0);
-        ++issued_v;
+        if (!mbar_wait(&emptyb[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) { ok = false; break; }
+        mbar_arrive_expect_tx(&fullb[bi], kTile);
+        tma_load_2d(smem + base + bi * kTile, &tm, &fullb[bi], col, kv0);
+        tma_load_2d(smem + base + bi * kTile + kHalf, &tm, &fullb[bi], col + 64, kv0);
+        ++issued;
       }
       if (!ok) {
         volatile int never = 0;
-        mbar_wait(q_full, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
-        for (uint32_t j = (issued_k > 2 ? issued_k - 2 : 0); j < issued_k; ++j)
-          mbar_wait(&k_full[j & 1], (j >> 1) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
-        for (uint32_t j = (issued_v > 2 ? issued_v - 2 : 0); j < issued_v; ++j)
-          mbar_wait(&v_full[j & 1], (j >> 1) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
+        if (kq) mbar_wait(q_full, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
+        for (uint32_t j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+          mbar_wait(&fullb[j & 1], (j >> 1) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
       }
     }
    } else if (warp == 9) {
@@ -317,7 +343,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           m_run = m_new;
           l *= alpha;
         }
-        // p = 2^(s * sl2 - m): packed FMA, MUFU exp2, packed row sums, bf16 pairs
+        // p = 2^(s * sl2 - m): packed FMA, exp2 on MUFU (5 of 8 pairs) or the FMA
+        // pipe (3 of 8), packed row sums, bf16 pairs
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm = f2_pack(-m_run, -m_run);
         uint64_t sum2[4] = {0, 0, 0, 0};
         uint32_t pw[64];
@@ -325,7 +352,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         for (int c = 0; c < 64; ++c) {
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2x2, negm), x0, x1);
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          float e0, e1;
+          if ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6) {  // 3 of 8 pairs on the FMA pipe
+            exp2_poly_pair(x0, x1, e0, e1);
+          } else {
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
+          }
           sum2[c & 3] = f2_add(sum2[c & 3], f2_pack(e0, e1));
           pw[c] = pack_bf16x2(e0, e1);
         }
