@@ -194,6 +194,16 @@ ZI_API int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int
                      const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, void* d_ws,
                      size_t ws_bytes, zi_stream_t stream);
 
+/* zi_model_forward that also copies the residual stream after every block into
+ * d_trace, fp32 [n_noise + n_ctx + n_main][rows][dim] in the library's row order
+ * (rows = batch * s_img image rows, then batch * s_txt text rows; blocks in
+ * execution order: noise refiners, context refiners, main blocks).  The kernels
+ * and their launch shapes are those of zi_model_forward; the copies are extra.
+ * Used to check every block of a full-size forward against a reference. */
+ZI_API int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w,
+                                  int s_txt, const float* d_latent, const float* d_t, const uint16_t* d_txt,
+                                  float* d_out, float* d_trace, void* d_ws, size_t ws_bytes, zi_stream_t stream);
+
 /* FlowMatch-Euler step in place (z-image-turbo-mnn "Scheduler"):
  *   y = d_out_uncond ? d_out_uncond + guidance (d_out_cond - d_out_uncond) : d_out_cond
  *   d_x += (sigma_next - sigma) * (-y)          (n fp32 elements)

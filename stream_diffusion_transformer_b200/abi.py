@@ -65,6 +65,9 @@ _SIGS = {
                                          c_int, c_void_p, c_void_p, c_void_p]),
     "zi_model_forward": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "zi_model_forward_trace": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                       c_void_p]),
     "zi_euler_step": (c_int, [c_void_p, c_void_p, c_void_p, c_float, c_double, c_double, c_size_t, c_void_p]),
     "zi_sigmas": (c_int, [c_int, c_double, POINTER(c_double)]),
     "zi_positions": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),

@@ -655,9 +655,10 @@ int zi_block_forward_noalloc(const zi_config* cfg, const zi_block_weights* w, co
                           stream);
 }
 
-int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
-                     const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, void* d_ws,
-                     size_t ws_bytes, zi_stream_t stream) {
+namespace {
+int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
+                       const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, float* d_trace,
+                       void* d_ws, size_t ws_bytes, zi_stream_t stream) {
   ZI_TRY(check_cfg(cfg));
   if (!w || !d_latent || !d_t || !d_txt || !d_out || batch <= 0 || lat_h <= 0 || lat_w <= 0 || s_txt <= 0)
     return ZI_ERR_ARG;
@@ -708,6 +709,14 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
   uint16_t* capn = reinterpret_cast<uint16_t*>(ws + L.capn);
   const RowMap map{rows_img, s_img, s_txt};
   const float eps = cfg->norm_eps;
+  int traced = 0;
+  auto trace = [&]() -> int {
+    if (!d_trace) return ZI_OK;
+    const size_t n = size_t(rows) * D;
+    if (cudaMemcpyAsync(d_trace + size_t(traced++) * n, x, n * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return ZI_ERR_CUDA;
+    return ZI_OK;
+  };
 
   // timestep conditioning and every adaLN projection
   {
@@ -810,6 +819,7 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
         if (i + 1 < cfg->n_noise) nx = NextNormSpec{NEXT_RMS, w->noise[i + 1].g_attn1, mod_of_noise(i + 1), 0};
         nx.next_rows = rows_img;
         ZI_TRY(run_block(b, nx, st));
+        ZI_TRY(trace());
       }
     } else {
       ZI_TRY(run_rms_mod<float>(b.x_in, rows_img, D, w->main[0].g_attn1, mod_of_main(0), mod_ld, map, 0, eps, b.h,
@@ -828,6 +838,7 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
         if (i + 1 < cfg->n_ctx) nx = NextNormSpec{NEXT_RMS, w->ctx[i + 1].g_attn1, nullptr, 0};
         nx.next_rows = rows_txt;
         ZI_TRY(run_block(b, nx, st));
+        ZI_TRY(trace());
       }
     } else {
       ZI_TRY(run_rms_mod<float>(b.x_in, rows_txt, D, w->main[0].g_attn1, mod_of_main(0), mod_ld, map, rows_img, eps,
@@ -848,6 +859,7 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
       NextNormSpec nx{NEXT_LAYERNORM, nullptr, final_scale, rows_img};
       if (i + 1 < cfg->n_main) nx = NextNormSpec{NEXT_RMS, w->main[i + 1].g_attn1, mod_of_main(i + 1), rows};
       ZI_TRY(run_block(b, nx, st));
+      ZI_TRY(trace());
     }
   }
   // final layer: LayerNorm(1 + scale) is already in h (image rows); linear + bias + unpatchify
@@ -862,6 +874,24 @@ int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch,
     ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, ZI_KERNEL_GEMM_FINAL, h, w->final_w, rows_img, 4 * cfg->in_ch, D, ef, st)));
   }
   return ZI_OK;
+}
+
+}  // namespace
+
+int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
+                     const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, void* d_ws,
+                     size_t ws_bytes, zi_stream_t stream) {
+  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, d_latent, d_t, d_txt, d_out, nullptr, d_ws, ws_bytes,
+                            stream);
+}
+
+int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w,
+                           int s_txt, const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out,
+                           float* d_trace, void* d_ws, size_t ws_bytes, zi_stream_t stream) {
+  if (!d_trace) return ZI_ERR_ARG;
+  if (!aligned16(d_trace)) return ZI_ERR_ALIGN;
+  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, d_latent, d_t, d_txt, d_out, d_trace, d_ws, ws_bytes,
+                            stream);
 }
 
 int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond, float guidance, double sigma,

@@ -155,6 +155,22 @@ class DiT:
         return out
 
 
+def forward_trace(dit: "DiT", latent: torch.Tensor, t: torch.Tensor, txt: torch.Tensor):
+    """DiT.forward that also returns the residual stream after every block:
+    (out, trace fp32 [n_blocks, rows, dim]) with rows = image rows then text rows."""
+    B, C, Hl, Wl = latent.shape
+    L = txt.shape[1]
+    cfg = dit.cfg
+    rows = B * ((Hl // 2) * (Wl // 2) + L)
+    n_blocks = cfg.n_noise + cfg.n_ctx + cfg.n_main
+    trace = torch.empty((n_blocks, rows, cfg.dim), dtype=torch.float32, device=latent.device)
+    out = torch.empty_like(latent)
+    ws = dit.workspace(B, Hl, Wl, L)
+    abi.call("zi_model_forward_trace", ctypes.byref(cfg), ctypes.byref(dit.weights), B, Hl, Wl, L, _p(latent), _p(t),
+             _p(txt), _p(out), _p(trace), _p(ws), ws.numel(), _stream())
+    return out, trace
+
+
 def block_forward(cfg: abi.ZiConfig, blk: DeviceBlock, c: Optional[torch.Tensor], pos: torch.Tensor,
                   x_in: torch.Tensor, x_out: Optional[torch.Tensor] = None,
                   ws: Optional[torch.Tensor] = None) -> torch.Tensor:

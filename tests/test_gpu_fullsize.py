@@ -1,0 +1,142 @@
+"""Full-size parity: the 4,128-token forward the benchmark times, checked block by block.
+
+The whole 34-block forward at 1024x1024 (4,096 image + 32 text tokens, t = 0.5,
+all 6,154,908,736 parameters) is too slow for the CPU oracle to redo in full, so
+the forward is run with zi_model_forward_trace (same kernels and launch shapes as
+zi_model_forward, plus a copy of the residual stream after every block) and every
+checked block is recomputed by the oracle from the GPU's own input to that block,
+for a sample of query rows (keys and values over the whole sequence).  The first
+refiner of each stream starts from the oracle's own embedding, and the final
+layer is checked on sampled tokens of the output.
+
+Bars: per block rel-L2 <= 2e-2, cosine >= 0.999, and update cosine >= 0.99 on the
+sampled rows (the block bar); final layer rel-L2 <= 2e-2, cosine >= 0.999.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from gpu_util import assert_parity, require_gpu, torch
+import zimage_inputs as zi
+from oracle import zimage_ref as ref
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+SEED = 0
+LAT = 128       # latent side of a 1024x1024 image
+S_TXT = 32
+T = 0.5
+
+
+@pytest.fixture(scope="module")
+def run():
+    require_gpu()
+    from stream_diffusion_transformer_b200 import abi, model
+    abi.lib()
+    abi.clear_device_status()
+    d = zi.FULL
+    threads = max(1, min(32, os.cpu_count() or 1))
+    dit = model.DiT(model.make_config(d), lambda keys: zi.make_weights(d, seed=SEED, keys=keys, threads=threads))
+    lat = zi.make_latent(d, 1, LAT, LAT, seed=SEED)
+    txt = zi.make_text(d, 1, S_TXT, seed=SEED)
+    t = np.array([T], dtype=np.float32)
+    lat_d = torch.from_numpy(lat).cuda()
+    t_d = torch.from_numpy(t).cuda()
+    txt_d = torch.from_numpy(txt.view(np.int16)).cuda().view(torch.bfloat16)
+    out_tr, trace = model.forward_trace(dit, lat_d, t_d, txt_d)
+    out = dit.forward(lat_d, t_d, txt_d)
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    res = dict(d=d, lat=lat, txt=txt, t=t, out=out.cpu().numpy(), out_tr=out_tr.cpu().numpy(),
+               trace=trace.cpu().numpy())
+    del dit, trace
+    torch.cuda.empty_cache()
+    s_img = (LAT // 2) ** 2
+    res["s_img"] = s_img
+    res["ang"] = ref.rope_angles(ref.position_ids(S_TXT, LAT // 2, LAT // 2), d.rope_axes)
+    top = ref.Weights(zi.make_weights(d, seed=SEED, keys=[k for k, _, _ in zi.weight_specs(d)
+                                                          if not k.startswith(("layers.", "noise_refiner.",
+                                                                               "context_refiner."))]))
+    res["top"] = top
+    res["c"] = ref.t_embed(t.astype(np.float64), top)[0]
+    rng = np.random.default_rng(5)
+    img_rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, 128, 2047, 2048, s_img - 2, s_img - 1],
+                                         rng.integers(0, s_img, 22)]))
+    res["img_rows"] = img_rows
+    res["all_rows"] = np.concatenate([img_rows, s_img + np.arange(S_TXT)])
+    return res
+
+
+def _block_weights(d, prefix, modulated):
+    keys = [k for k, _, _ in zi.block_specs(prefix, d, modulated)]
+    return ref.Weights(zi.make_weights(d, seed=SEED, keys=keys, threads=8))
+
+
+def _check(got_rows, want_rows, x_rows, what):
+    assert_parity(got_rows, want_rows, rel=2e-2, cos=0.999, what=what)
+    assert_parity(got_rows - x_rows, want_rows - x_rows, rel=1.0, cos=0.99, what=what + " update")
+
+
+def test_traced_run_is_the_timed_forward(run):
+    """The trace copies do not change the computation: outputs are bit-identical."""
+    np.testing.assert_array_equal(run["out_tr"], run["out"])
+    assert np.all(np.isfinite(run["out"]))
+
+
+def test_first_noise_refiner_from_oracle_embedding(run):
+    d, s_img = run["d"], run["s_img"]
+    x0 = ref.linear(ref.patchify(run["lat"].astype(np.float64))[0], run["top"]("x_embedder.weight"),
+                    run["top"]("x_embedder.bias"))
+    W = _block_weights(d, "noise_refiner.0", True)
+    rows = run["img_rows"]
+    want = ref.block_forward_rows(x0, W, "noise_refiner.0", d, run["ang"][:s_img], run["c"], rows)
+    _check(run["trace"][0][rows], want, x0[rows], "noise_refiner.0")
+
+
+def test_first_context_refiner_from_oracle_embedding(run):
+    d, s_img = run["d"], run["s_img"]
+    xt = ref.embed_text(zi.bf16_bits_to_f32(run["txt"])[0].astype(np.float64), run["top"])
+    W = _block_weights(d, "context_refiner.0", False)
+    rows = np.arange(S_TXT)
+    want = ref.block_forward_rows(xt, W, "context_refiner.0", d, run["ang"][s_img:], None, rows)
+    k = d.n_noise  # trace index of context_refiner.0
+    _check(run["trace"][k][s_img + rows], want, xt, "context_refiner.0")
+
+
+@pytest.mark.parametrize("which", ["noise_refiner.1", "context_refiner.1", "layers.0", "layers.1", "layers.14",
+                                   "layers.29"])
+def test_block_on_gpu_input(run, which):
+    d, s_img = run["d"], run["s_img"]
+    kind, idx = which.split(".")
+    idx = int(idx)
+    order = ([f"noise_refiner.{i}" for i in range(d.n_noise)] + [f"context_refiner.{i}" for i in range(d.n_ctx)]
+             + [f"layers.{i}" for i in range(d.n_main)])
+    k = order.index(which)
+    if kind == "noise_refiner":
+        x_in = run["trace"][k - 1][:s_img].astype(np.float64)
+        ang, c, rows, off = run["ang"][:s_img], run["c"], run["img_rows"], 0
+    elif kind == "context_refiner":
+        x_in = run["trace"][k - 1][s_img:].astype(np.float64)
+        ang, c, rows, off = run["ang"][s_img:], None, np.arange(S_TXT), s_img
+    else:
+        x_in = run["trace"][k - 1].astype(np.float64)
+        ang, c, rows, off = run["ang"], run["c"], run["all_rows"], 0
+    W = _block_weights(d, which, c is not None)
+    want = ref.block_forward_rows(x_in, W, which, d, ang, c, rows)
+    _check(run["trace"][k][off + rows], want, x_in[rows], which)
+
+
+def test_final_layer_on_sampled_tokens(run):
+    d, s_img = run["d"], run["s_img"]
+    rows = run["img_rows"]
+    x_last = run["trace"][-1][rows].astype(np.float64)
+    y = ref.final_layer(x_last, run["top"], run["c"])  # [n, 64], feature (i*2 + j)*16 + channel
+    gw = LAT // 2
+    got = np.empty_like(y)
+    for n, r in enumerate(rows):
+        ty, tx = divmod(int(r), gw)
+        for f in range(64):
+            ch, pq = f % 16, f // 16
+            got[n, f] = run["out"][0, ch, 2 * ty + (pq >> 1), 2 * tx + (pq & 1)]
+    assert_parity(got, y, rel=2e-2, cos=0.999, what="final layer")
