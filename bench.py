@@ -428,6 +428,38 @@ def run_block_workload(args):
                       "kernels": prof.by_kernel(), "device_status": abi.device_status()}), flush=True)
 
 
+def run_loop_workload(args, n_steps: int = 8, s_txt: int = 128):
+    """The 8-step Turbo loop: 8 forwards at 4,096 image + 128 text tokens with the
+    FlowMatch-Euler step (shift 3) between them; each timed step is one whole loop."""
+    import torch
+
+    from stream_diffusion_transformer_b200 import abi, model
+
+    d = zi.FULL
+    threads = max(1, min(32, (os.cpu_count() or 8)))
+    dit = model.DiT(model.make_config(d), lambda keys: zi.make_weights(d, seed=SEED, keys=keys, threads=threads))
+    lat = torch.from_numpy(zi.make_latent(d, 1, LAT_H, LAT_W, seed=SEED)).cuda()
+    txt = torch.from_numpy(zi.make_text(d, 1, s_txt, seed=SEED).view(np.int16)).cuda().view(torch.bfloat16)
+    for _ in range(args.warmup):
+        dit.denoise(lat, txt, n_steps=n_steps)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        e0.record()
+        for _ in range(args.steps):
+            x = dit.denoise(lat, txt, n_steps=n_steps)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    s_img = (LAT_H // 2) * (LAT_W // 2)
+    fl = n_steps * forward_flops(d, s_img, s_txt)
+    print(json.dumps({"workload": f"8-step Turbo loop, 1024x1024, {s_img} + {s_txt} tokens, shift 3",
+                      "ms_per_loop": ms, "ms_per_forward": ms / n_steps, "value": fl / (ms * 1e-3) / 1e12,
+                      "unit": "TFLOP/s", "steps": args.steps, "warmup": args.warmup,
+                      "finite": bool(torch.isfinite(x).all().item()), "device_status": abi.device_status(),
+                      "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,12 +467,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["forward", "block"], default="forward",
+    ap.add_argument("--workload", choices=["forward", "block", "turbo8"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
-                         "(a profiling-sized case)")
+                         "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens")
     args = ap.parse_args()
     if args.workload == "block":
         run_block_workload(args)
+        return
+    if args.workload == "turbo8":
+        run_loop_workload(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

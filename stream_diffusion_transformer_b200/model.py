@@ -140,6 +140,35 @@ class DiT:
             self._ws[key] = torch.empty(n, dtype=torch.uint8, device=self.device)
         return self._ws[key]
 
+    def denoise(self, latent: torch.Tensor, txt: torch.Tensor, n_steps: int = 8, shift: float = 3.0,
+                guidance: Optional[float] = None, txt_uncond: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """FlowMatch-Euler loop (z-image-turbo-mnn "Scheduler"): n_steps forwards at
+        t = 1 - sigma'_i, each followed by zi_euler_step with sigma'_i -> sigma'_{i+1};
+        with guidance and txt_uncond, the conditional and unconditional branches run
+        as one batch-2 forward and are combined y_u + g (y_c - y_u).  Returns the
+        final latent (a new tensor; `latent` is left unchanged)."""
+        sig = abi.sigmas(n_steps, shift)
+        x = latent.clone()
+        B = x.shape[0]
+        cfg_mode = guidance is not None and txt_uncond is not None
+        out = torch.empty((2 * B,) + tuple(x.shape[1:]) if cfg_mode else x.shape, dtype=torch.float32,
+                          device=x.device)
+        tt = torch.empty(2 * B if cfg_mode else B, dtype=torch.float32, device=x.device)
+        txt_all = torch.cat([txt, txt_uncond], 0) if cfg_mode else txt
+        x_in = torch.empty((2 * B,) + tuple(x.shape[1:]), dtype=torch.float32, device=x.device) if cfg_mode else x
+        for i in range(n_steps):
+            tt.fill_(1.0 - sig[i])
+            if cfg_mode:
+                x_in[:B].copy_(x)
+                x_in[B:].copy_(x)
+            self.forward(x_in, tt, txt_all, out)
+            if cfg_mode:
+                abi.call("zi_euler_step", _p(x), _p(out[:B]), _p(out[B:]), float(guidance), sig[i], sig[i + 1],
+                         x.numel(), _stream())
+            else:
+                abi.call("zi_euler_step", _p(x), _p(out), None, 0.0, sig[i], sig[i + 1], x.numel(), _stream())
+        return x
+
     def forward(self, latent: torch.Tensor, t: torch.Tensor, txt: torch.Tensor,
                 out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
         """latent fp32 [B, C, H/8, W/8], t fp32 [B] (1 = clean), txt bf16 [B, L, cap_dim] -> raw output."""

@@ -42,6 +42,7 @@ def cosine(got, want) -> float:
 
 def assert_parity(got, want, rel=2e-2, cos=0.999, what=""):
     r, c = rel_l2(got, want), cosine(got, want)
+    print(f"[parity] {what}: rel-L2 {r:.3e} cos {c:.7f}")
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     assert r <= rel and c >= cos, f"{what}: rel-L2 {r:.3e} (<= {rel}), cos {c:.6f} (>= {cos})"
     return r, c

@@ -58,3 +58,42 @@ def test_full_width_shallow_model():
     d = dataclasses.replace(zi.FULL, n_noise=1, n_ctx=1, n_main=2)
     got, want = run_model(d, 1, 32, 32, 32, [0.25], seed=2)
     assert_parity(got, want, rel=3e-2, cos=0.995, what="full-width shallow model")
+
+
+def _denoise_case(d, lat_hw, s_txt, n_steps, seed, guidance=None):
+    from stream_diffusion_transformer_b200 import model
+    from oracle import scheduler_ref as sch
+    bits = zi.make_weights(d, seed=seed)
+    dit = model.DiT(model.make_config(d), lambda keys: {k: bits[k] for k in keys})
+    lat = zi.make_latent(d, 1, lat_hw, lat_hw, seed=seed)
+    txt = zi.make_text(d, 1, s_txt, seed=seed)
+    txt_u = zi.make_text(d, 1, s_txt, seed=seed, uncond=True)
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    got = dit.denoise(torch.from_numpy(lat).cuda(), dev(txt), n_steps=n_steps, shift=3.0, guidance=guidance,
+                      txt_uncond=dev(txt_u) if guidance is not None else None)
+    torch.cuda.synchronize()
+    W = ref.Weights(bits)
+    tc = zi.bf16_bits_to_f32(txt).astype(np.float64)
+    tu = zi.bf16_bits_to_f32(txt_u).astype(np.float64)
+
+    def model_fn(x, t, uncond):
+        return ref.model_forward(x, t, tu if uncond else tc, W, d)
+
+    want = sch.denoise(lat.astype(np.float64), model_fn, n_steps, 3.0, guidance)
+    return got.cpu().numpy().astype(np.float64), want, lat.astype(np.float64)
+
+
+def test_turbo_loop_8_steps():
+    """8-step FlowMatch-Euler loop (shift 3, t = 1 - sigma', output negated) at full width,
+    1 + 1 + 2 blocks, 256 image + 128 text tokens; final latent against the oracle's loop."""
+    d = dataclasses.replace(zi.FULL, n_noise=1, n_ctx=1, n_main=2)
+    got, want, x0 = _denoise_case(d, 32, 128, 8, seed=3)
+    assert_parity(got, want, rel=3e-2, cos=0.995, what="8-step loop final latent")
+    assert_parity(got - x0, want - x0, rel=3e-2, cos=0.995, what="8-step loop latent change")
+
+
+def test_cfg_loop_batch2():
+    """Guidance 4: conditional and unconditional texts as one batch-2 forward per step."""
+    got, want, x0 = _denoise_case(zi.TINY_R, 8, 16, 4, seed=4, guidance=4.0)
+    assert_parity(got, want, rel=3e-2, cos=0.995, what="CFG loop final latent")
+    assert_parity(got - x0, want - x0, rel=3e-2, cos=0.995, what="CFG loop latent change")
