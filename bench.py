@@ -201,6 +201,42 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def make_fetch(d: zi.Dims, rank: int, world: int, device, threads: int):
+    """fetch(keys) -> {key: bf16 bits}: rank 0 draws the seeded weights on its host
+    threads and broadcasts them (over the process group's backend) to the other
+    ranks, so every replica holds identical weights and the host draws them once."""
+    import torch
+    import torch.distributed as dist
+
+    specs = {k: s for k, s, _ in zi.weight_specs(d)}
+
+    def fetch(keys):
+        out = zi.make_weights(d, seed=SEED, keys=keys, threads=threads) if rank == 0 or world == 1 else {}
+        if world == 1:
+            return out
+        res = {}
+        for k in keys:  # as raw bytes: neither NCCL nor gloo reduces or broadcasts 16-bit integers
+            n = int(np.prod(specs[k])) * 2
+            t = (torch.from_numpy(np.ascontiguousarray(out[k]).reshape(-1).view(np.uint8)).to(device) if rank == 0
+                 else torch.empty(n, dtype=torch.uint8, device=device))
+            dist.broadcast(t, 0)
+            res[k] = t.cpu().numpy().view(np.uint16).reshape(specs[k])
+        return res
+
+    return fetch
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (each rank timed its own device)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -219,21 +255,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # weights: generated on rank 0's host threads, broadcast to the other ranks
     threads = max(1, min(32, (os.cpu_count() or 8)))
 
-    def fetch(keys):
-        if world == 1 or rank == 0:
-            out = zi.make_weights(d, seed=SEED, keys=keys, threads=threads)
-        else:
-            out = {}
-        if world > 1:
-            specs = {k: s for k, s, _ in zi.weight_specs(d)}
-            res = {}
-            for k in keys:
-                t = (torch.from_numpy(out[k].view(np.int16)).to(dev) if rank == 0
-                     else torch.empty(specs[k], dtype=torch.int16, device=dev))
-                dist.broadcast(t, 0)
-                res[k] = t.cpu().numpy().view(np.uint16)
-            return res
-        return out
+    fetch = make_fetch(d, rank, world, dev, threads)
 
     t_load = time.perf_counter()
     dit = model.DiT(cfg, fetch, device=dev)
@@ -265,11 +287,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             end.record(stream)
             torch.cuda.synchronize()
         barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
     status = abi.device_status()
     if status != 0:
         raise RuntimeError(f"device pipeline timeout (code {status}) during the timed region")
@@ -298,11 +316,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     h2d = h_lat.numel() * 4 + h_txt.numel() * 2 + h_t.numel() * 4
     d2h = h_out.numel() * 4
 
