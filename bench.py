@@ -474,6 +474,54 @@ def run_loop_workload(args, n_steps: int = 8, s_txt: int = 128):
                       "clocks": clocks.summary()}), flush=True)
 
 
+def run_cfg_workload(args):
+    """One classifier-free-guidance step at 2048x2048: a batch-2 forward (conditional
+    and unconditional text, 16,384 image + 512 text tokens each) and the guidance-4
+    combine inside the Euler update."""
+    import torch
+
+    from stream_diffusion_transformer_b200 import abi, model
+
+    d = zi.FULL
+    lat_hw, s_txt = 256, 512
+    threads = max(1, min(32, (os.cpu_count() or 8)))
+    dit = model.DiT(model.make_config(d), lambda keys: zi.make_weights(d, seed=SEED, keys=keys, threads=threads))
+    lat1 = torch.from_numpy(zi.make_latent(d, 1, lat_hw, lat_hw, seed=SEED)).cuda()
+    lat = torch.cat([lat1, lat1], 0).contiguous()
+    txt = torch.cat([torch.from_numpy(zi.make_text(d, 1, s_txt, seed=SEED).view(np.int16)),
+                     torch.from_numpy(zi.make_text(d, 1, s_txt, seed=SEED, uncond=True).view(np.int16))],
+                    0).cuda().view(torch.bfloat16).contiguous()
+    tt = torch.full((2,), T_VALUE, dtype=torch.float32, device="cuda")
+    out = torch.empty_like(lat)
+    x = lat1.clone()
+    sig = abi.sigmas(8, 3.0)
+
+    def step():
+        dit.forward(lat, tt, txt, out)
+        abi.call("zi_euler_step", model._p(x), model._p(out[:1]), model._p(out[1:]), 4.0, sig[0], sig[1],
+                 x.numel(), model._stream())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks, abi.Profile(capacity=300 * args.steps + 16) as prof:
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    s_img = (lat_hw // 2) ** 2
+    fl = forward_flops(d, s_img, s_txt, batch=2)
+    by = {k: {"launches": v[0], "ms": round(v[1] / args.steps, 3)} for k, v in prof.by_kernel().items()}
+    print(json.dumps({"workload": f"CFG step, 2048x2048, batch 2 x ({s_img} + {s_txt}) tokens, guidance 4",
+                      "ms_per_step": ms, "value": fl / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "flops_per_step": fl, "steps": args.steps, "warmup": args.warmup, "kernels_ms_per_step": by,
+                      "finite": bool(torch.isfinite(x).all().item()), "device_status": abi.device_status(),
+                      "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,15 +529,19 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["forward", "block", "turbo8"], default="forward",
+    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
-                         "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens")
+                         "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens; "
+                         "cfg: one guidance step at 2048x2048, batch 2 x 16,896 tokens")
     args = ap.parse_args()
     if args.workload == "block":
         run_block_workload(args)
         return
     if args.workload == "turbo8":
         run_loop_workload(args)
+        return
+    if args.workload == "cfg":
+        run_cfg_workload(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -68,3 +68,32 @@ def test_full_width_unmodulated_text_block():
     """A context-refiner-shaped block on 32 text tokens only (a single partial tile)."""
     d = dataclasses.replace(zi.FULL, n_noise=0, n_ctx=1, n_main=1)
     run_block(d, "context_refiner.0", False, 1, 32, 0, 0, seed=4)
+
+
+@pytest.mark.slow
+def test_full_width_block_cfg_batch2_16896_tokens():
+    """A main block of the CFG workload: batch 2 x (16,384 image + 512 text) tokens, on
+    sampled rows (keys and values over the whole 16,896-token sequence of each element)."""
+    from stream_diffusion_transformer_b200 import model
+    d = dataclasses.replace(zi.FULL, n_noise=0, n_ctx=0, n_main=1)
+    cfg = model.make_config(d)
+    keys = model.block_keys("layers.0", True)
+    bits = zi.make_weights(d, seed=7, keys=keys, threads=8)
+    s_txt, gh, gw = 512, 128, 128
+    S = gh * gw + s_txt
+    x = zi.make_stream(d, 2, S, seed=7)
+    c = zi.make_cond(d, 2, seed=7)
+    blk = model.DeviceBlock(cfg, "layers.0", bits, True, "cuda")
+    pos = model.positions(s_txt, gh, gw)
+    out = model.block_forward(cfg, blk, torch.from_numpy(c).cuda(), pos, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    W = ref.Weights(bits)
+    ang = ref.rope_angles(ref.position_ids(s_txt, gh, gw), d.rope_axes)
+    rows = np.unique(np.concatenate([[0, 127, 128, 8191, 16383, 16384, S - 1],
+                                     np.random.default_rng(7).integers(0, S, 17)]))
+    for b in range(2):
+        want = ref.block_forward_rows(x[b].astype(np.float64), W, "layers.0", d, ang, c[b].astype(np.float64), rows)
+        assert_parity(got[b][rows], want, rel=2e-2, cos=0.999, what=f"CFG-size block b={b}")
+        assert_parity(got[b][rows] - x[b][rows], want - x[b][rows], rel=1.0, cos=0.99,
+                      what=f"CFG-size block delta b={b}")
