@@ -126,6 +126,8 @@ typedef struct zi_model_weights {
   const zi_block_weights* noise; /* host array [n_noise], modulated */
   const zi_block_weights* ctx;   /* host array [n_ctx], w_ada == NULL */
   const zi_block_weights* main;  /* host array [n_main], modulated */
+  const uint16_t* cap_pad;   /* [D] cap_pad_token: embedding of padded text rows
+                                (read by zi_model_forward_varlen only; may be NULL otherwise) */
 } zi_model_weights;
 
 /* Human-readable text of a status code (static storage). */
@@ -159,8 +161,8 @@ ZI_API int zi_pack_ffn(const uint16_t* w1, const uint16_t* w3, const uint16_t* w
 /* Bytes of workspace zi_block_forward needs for batch x seq tokens. */
 ZI_API int zi_block_workspace_size(const zi_config* cfg, int batch, int seq, size_t* h_bytes);
 
-/* Bytes of workspace zi_model_forward needs for batch x (s_img + s_txt) tokens,
- * s_img = (lat_h/2)(lat_w/2). */
+/* Bytes of workspace zi_model_forward (and zi_model_forward_varlen) needs for
+ * batch x (s_img + s_txt) tokens, s_img = (lat_h/2)(lat_w/2). */
 ZI_API int zi_model_workspace_size(const zi_config* cfg, int batch, int lat_h, int lat_w, int s_txt, size_t* h_bytes);
 
 /* ---------------------------------------------------------------- the forward */
@@ -189,10 +191,32 @@ ZI_API int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, con
  * Sequence per batch element: [(lat_h/2)(lat_w/2) image tokens; s_txt text tokens],
  * image tokens refined by the noise refiners, text tokens by the context
  * refiners, then all tokens through the main blocks and image tokens through
- * the final layer.  s_txt >= 1; no padding is added (pad tokens unused). */
+ * the final layer.  s_txt >= 1; every text row is a real token (no padding;
+ * for a batch of prompts of different lengths use zi_model_forward_varlen). */
 ZI_API int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
                      const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, void* d_ws,
                      size_t ws_bytes, zi_stream_t stream);
+
+/* zi_model_forward for a batch whose prompts differ in length (FastVideo zimage
+ * handoff, "Transformer": a padded variable-length stream needs a key mask;
+ * ostris "Z-Image", "Architecture": the checkpoint's cap_pad_token).  Element b
+ * holds h_txt_len[b] real text tokens followed by s_txt - h_txt_len[b] padding
+ * rows of d_txt (their contents are ignored):
+ *   - padding rows take w->cap_pad as their embedding (after the cap embedder);
+ *   - padding rows are removed from the keys of every attention (context
+ *     refiners and main blocks), i.e. an additive -inf key mask; the image rows
+ *     and real text rows then see exactly their unpadded sequence;
+ *   - positions follow each element's own length: image token (r, c) ->
+ *     (h_txt_len[b] + 1, r, c), text row j -> (j + 1, 0, 0) (a reading; it makes
+ *     the output for element b equal to a batch-1 forward on its unpadded text).
+ *   h_txt_len  HOST int32 [batch], each in [1, s_txt]; otherwise ZI_ERR_ARG.
+ * Other arguments as for zi_model_forward; w->cap_pad must be non-NULL.  The
+ * lengths reach the device as kernel arguments (no host-to-device copy), so the
+ * call can be captured in a CUDA graph. */
+ZI_API int zi_model_forward_varlen(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w,
+                                   int s_txt, const int32_t* h_txt_len, const float* d_latent, const float* d_t,
+                                   const uint16_t* d_txt, float* d_out, void* d_ws, size_t ws_bytes,
+                                   zi_stream_t stream);
 
 /* zi_model_forward that also copies the residual stream after every block into
  * d_trace, fp32 [n_noise + n_ctx + n_main][rows][dim] in the library's row order
@@ -274,6 +298,13 @@ ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c,
  * d_out bf16 [batch*seq, heads*128]. */
 ZI_API int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads, zi_stream_t stream);
 
+/* zi_attention with a key mask: element b attends to its first d_kv_len[b] keys
+ * only (rows past them are padding; FastVideo zimage handoff, "Transformer").
+ * Every query row is still computed.  d_kv_len DEVICE int32 [batch]; values
+ * are clamped to [1, seq] on the device. */
+ZI_API int zi_attention_varlen(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads,
+                               const int32_t* d_kv_len, zi_stream_t stream);
+
 /* ---------------------------------------------------------------- launch profiling */
 
 /* Kernel identities reported by zi_profile_end. */
@@ -293,7 +324,8 @@ enum zi_kernel_kind {
   ZI_KERNEL_GEMM_EMBED = 13,    /* x_embedder / cap_embedder projection */
   ZI_KERNEL_GEMM_FINAL = 14,    /* final linear + unpatchify */
   ZI_KERNEL_EULER = 15,         /* Euler / CFG step */
-  ZI_KERNEL_GEMM = 16           /* zi_gemm_bf16 */
+  ZI_KERNEL_GEMM = 16,          /* zi_gemm_bf16 */
+  ZI_KERNEL_TEXT_PAD = 17       /* cap_pad_token into padded text rows */
 };
 
 /* Start recording launch timings on this host thread: from the next kernel the

@@ -130,6 +130,17 @@ def position_ids(s_txt: int, grid_h: int, grid_w: int) -> np.ndarray:
     return np.concatenate([img, txt], axis=0).astype(np.int32)
 
 
+def position_ids_varlen(s_txt: int, txt_len: int, grid_h: int, grid_w: int) -> np.ndarray:
+    """Positions of one padded sequence [image; txt_len text tokens; s_txt - txt_len pads].
+
+    Reading for padded batches: positions follow the element's own text length,
+    so image token (r, c) -> (txt_len + 1, r, c); text and pad row j -> (j + 1, 0, 0).
+    With the pads masked as keys this makes padding invisible to the valid tokens."""
+    pos = position_ids(s_txt, grid_h, grid_w)
+    pos[:grid_h * grid_w, 0] = txt_len + 1
+    return pos
+
+
 def rope_angles(pos: np.ndarray, axes=(32, 48, 48), theta: float = ROPE_THETA) -> np.ndarray:
     """Rotation angles [S, sum(axes)/2]: axis a, pair j -> pos[:, a] * theta^(-2j/d_a)."""
     cols = []
@@ -150,13 +161,19 @@ def apply_rope(x: np.ndarray, angles: np.ndarray) -> np.ndarray:
     return np.stack([a * cs - b * sn, a * sn + b * cs], axis=-1).reshape(S, H, hd)
 
 
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
-    """Non-causal softmax(q k^T / sqrt(hd)) v per head; q, k, v [S, H, hd]."""
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_valid: Optional[np.ndarray] = None) -> np.ndarray:
+    """Non-causal softmax(q k^T / sqrt(hd)) v per head; q, k, v [S, H, hd].
+
+    key_valid (bool [T], optional): keys marked False are excluded (an additive
+    -inf key mask, FastVideo zimage handoff, "Transformer": the padded
+    variable-length stream needs a key mask)."""
     S, H, hd = q.shape
     out = np.empty((q.shape[0], H, hd), dtype=q.dtype)
     scale = 1.0 / np.sqrt(hd)
     for h in range(H):
         s = (q[:, h] @ k[:, h].T) * scale
+        if key_valid is not None:
+            s = np.where(key_valid[None, :], s, -np.inf)
         s = s - s.max(axis=1, keepdims=True)
         p = np.exp(s)
         p = p / p.sum(axis=1, keepdims=True)
@@ -174,7 +191,8 @@ def adaln(c: np.ndarray, W: Weights, prefix: str):
 
 
 def block_forward(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: np.ndarray,
-                  c: Optional[np.ndarray] = None, return_parts: bool = False):
+                  c: Optional[np.ndarray] = None, return_parts: bool = False,
+                  key_valid: Optional[np.ndarray] = None):
     """One S3-DiT block on x [S, D].  c=None runs the unmodulated (context-refiner) form.
 
     attention sublayer: h = RMSNorm1(x)(1 + scale_msa); q, k, v = h Wq, h Wk, h Wv;
@@ -197,7 +215,7 @@ def block_forward(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: np.nd
     v = linear(h, W(f"{a}.to_v.weight")).reshape(S, H, hd)
     q = apply_rope(rms_norm(q, W(f"{a}.norm_q.weight")), angles)
     k = apply_rope(rms_norm(k, W(f"{a}.norm_k.weight")), angles)
-    att = attention(q, k, v).reshape(S, D)
+    att = attention(q, k, v, key_valid).reshape(S, D)
     o = linear(att, W(f"{a}.to_out.weight"))
     x1 = x + gate_msa * rms_norm(o, W(f"{prefix}.attention_norm2.weight"))
     h2 = rms_norm(x1, W(f"{prefix}.ffn_norm1.weight")) * (1.0 + scale_mlp)
@@ -211,7 +229,8 @@ def block_forward(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: np.nd
 
 
 def block_forward_rows(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: np.ndarray,
-                       c: Optional[np.ndarray], rows: np.ndarray) -> np.ndarray:
+                       c: Optional[np.ndarray], rows: np.ndarray,
+                       key_valid: Optional[np.ndarray] = None) -> np.ndarray:
     """block_forward(x, ...)[rows], computed for those query rows only.
 
     Keys and values come from every row of x (the attention is over the whole
@@ -232,7 +251,7 @@ def block_forward_rows(x: np.ndarray, W: Weights, prefix: str, d: Dims, angles: 
     hr = h[rows]
     q = linear(hr, W(f"{a}.to_q.weight")).reshape(len(rows), H, hd)
     q = apply_rope(rms_norm(q, W(f"{a}.norm_q.weight")), angles[rows])
-    att = attention(q, k, v).reshape(len(rows), D)
+    att = attention(q, k, v, key_valid).reshape(len(rows), D)
     o = linear(att, W(f"{a}.to_out.weight"))
     x1 = x[rows] + gate_msa * rms_norm(o, W(f"{prefix}.attention_norm2.weight"))
     h2 = rms_norm(x1, W(f"{prefix}.ffn_norm1.weight")) * (1.0 + scale_mlp)
@@ -256,13 +275,17 @@ def embed_text(txt: np.ndarray, W: Weights) -> np.ndarray:
 
 
 def model_forward(latent: np.ndarray, t: np.ndarray, txt: np.ndarray, W: Weights, d: Dims,
-                  trace: Optional[list] = None) -> np.ndarray:
+                  trace: Optional[list] = None, txt_len: Optional[np.ndarray] = None) -> np.ndarray:
     """Full transformer forward.
 
     latent [B, C, H/8, W/8] (any float), t [B] in [0, 1] (1 = clean),
     txt [B, L, cap_dim] float.  Returns the raw model output [B, C, H/8, W/8]
     (the scheduler negates it).  ``trace``, if given, receives the residual
     stream [S, D] of sample 0 after every block, in execution order.
+
+    txt_len [B] (optional): element b has txt_len[b] valid text tokens; its text
+    rows from txt_len[b] on are padding: their embeddings are replaced by the
+    cap_pad_token and they are masked as keys in every attention.
     """
     B, C, Hl, Wl = latent.shape
     p = d.patch
@@ -271,23 +294,32 @@ def model_forward(latent: np.ndarray, t: np.ndarray, txt: np.ndarray, W: Weights
     L = txt.shape[1]
     tokens = patchify(np.asarray(latent, dtype=W.dtype), p)
     c_all = t_embed(t, W)
-    ang = rope_angles(position_ids(L, gh, gw), d.rope_axes)
     outs = []
     for b in range(B):
         c = c_all[b]
+        lb = L if txt_len is None else int(txt_len[b])
+        if txt_len is None:
+            ang = rope_angles(position_ids(L, gh, gw), d.rope_axes)
+            kv_txt = kv_all = None
+        else:
+            ang = rope_angles(position_ids_varlen(L, lb, gh, gw), d.rope_axes)
+            kv_txt = np.arange(L) < lb
+            kv_all = np.concatenate([np.ones(s_img, dtype=bool), kv_txt])
         xi = linear(tokens[b], W("x_embedder.weight"), W("x_embedder.bias"))
         xt = embed_text(np.asarray(txt[b], dtype=W.dtype), W)
+        if txt_len is not None and lb < L:
+            xt[lb:] = W("cap_pad_token")
         for i in range(d.n_noise):
             xi = block_forward(xi, W, f"noise_refiner.{i}", d, ang[:s_img], c)
             if trace is not None and b == 0:
                 trace.append(xi.copy())
         for i in range(d.n_ctx):
-            xt = block_forward(xt, W, f"context_refiner.{i}", d, ang[s_img:], None)
+            xt = block_forward(xt, W, f"context_refiner.{i}", d, ang[s_img:], None, key_valid=kv_txt)
             if trace is not None and b == 0:
                 trace.append(xt.copy())
         x = np.concatenate([xi, xt], axis=0)
         for i in range(d.n_main):
-            x = block_forward(x, W, f"layers.{i}", d, ang, c)
+            x = block_forward(x, W, f"layers.{i}", d, ang, c, key_valid=kv_all)
             if trace is not None and b == 0:
                 trace.append(x.copy())
         y = final_layer(x[:s_img], W, c)

@@ -47,7 +47,8 @@ MODEL_FIELDS = ("x_emb_w", "x_emb_b", "cap_norm", "cap_w", "cap_b", "t_w1", "t_b
 
 class ZiModelWeights(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in MODEL_FIELDS] + [
-        ("noise", POINTER(ZiBlockWeights)), ("ctx", POINTER(ZiBlockWeights)), ("main", POINTER(ZiBlockWeights))]
+        ("noise", POINTER(ZiBlockWeights)), ("ctx", POINTER(ZiBlockWeights)), ("main", POINTER(ZiBlockWeights)),
+        ("cap_pad", c_void_p)]
 
 
 _SIGS = {
@@ -65,6 +66,9 @@ _SIGS = {
                                          c_int, c_void_p, c_void_p, c_void_p]),
     "zi_model_forward": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "zi_model_forward_varlen": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
+                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                        c_void_p]),
     "zi_model_forward_trace": (c_int, [POINTER(ZiConfig), POINTER(ZiModelWeights), c_int, c_int, c_int, c_int,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                        c_void_p]),
@@ -74,6 +78,7 @@ _SIGS = {
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
     "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_attention_varlen": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_profile_begin": (c_int, [c_int]),
     "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),
     "zi_device_status": (c_int, [POINTER(c_int)]),
@@ -157,7 +162,7 @@ KERNEL_NAMES = {
     1: "gemm_qkv_qknorm_rope", 2: "attention", 3: "gemm_out_proj", 4: "gemm_ffn_up_swiglu",
     5: "gemm_ffn_down", 6: "post_norm_residual", 7: "pre_norm", 8: "adaln_gemv", 9: "timestep_mlp",
     10: "rope_table", 11: "positions", 12: "patchify", 13: "gemm_embed", 14: "gemm_final_unpatchify",
-    15: "euler", 16: "gemm",
+    15: "euler", 16: "gemm", 17: "text_pad",
 }
 
 

@@ -21,7 +21,9 @@
 // from the same columns; the tensor core executes one CTA's MMAs in issue order.
 // The key sequence of a batch element can be split over two row segments of
 // the token buffer (image rows and text rows); key tiles that run past a
-// segment's end are masked to -inf.
+// segment's end are masked to -inf.  An optional per-element key count for the
+// last segment (kv_len) drops that segment's trailing rows (padding) from the
+// keys: tiles wholly past it are never loaded, the tile it ends in is masked.
 #pragma once
 #include "zi_common.cuh"
 
@@ -36,6 +38,7 @@ struct AttnParams {
   int seg_len[2];   // rows per batch element in segment i (element b starts at row0 + b * len)
   int q_tiles;      // query tiles per batch element (both segments)
   float scale_log2; // log2(e) / sqrt(head_dim)
+  const int* kv_len;  // [batch] keys of the last segment per element, or null (= its seg_len)
 };
 
 namespace attn {
@@ -50,7 +53,18 @@ constexpr uint32_t kSmemBytes = kBar + 256 + 1024;
 constexpr uint32_t kColS = 0, kColO = 256;  // S_t at kColS + 128 t, O_t at kColO + 128 t
 }  // namespace attn
 
-ZI_DEV void attn_tile_rows(const AttnParams& p, int b, int tile, int& row0, int& valid) {
+// Keys of the last segment of element b: kv_len[b] clamped to [1, seg_len], or all.
+ZI_DEV int attn_last_len(const AttnParams& p) { return p.nseg > 1 ? p.seg_len[1] : p.seg_len[0]; }
+
+ZI_DEV int attn_last_keys(const AttnParams& p, int b) {
+  const int n = attn_last_len(p);
+  if (!p.kv_len) return n;
+  return max(1, min(n, p.kv_len[b]));
+}
+
+// Rows of tile `tile` of element b; the last segment counts last_n rows (all of
+// them for query tiles, the element's key count for key tiles).
+ZI_DEV void attn_tile_rows(const AttnParams& p, int b, int tile, int last_n, int& row0, int& valid) {
   int seg = 0;
   int t = tile;
   const int n0 = (p.seg_len[0] + 127) / 128;
@@ -58,8 +72,11 @@ ZI_DEV void attn_tile_rows(const AttnParams& p, int b, int tile, int& row0, int&
     seg = 1;
     t -= n0;
   }
-  row0 = p.seg_row0[seg] + b * p.seg_len[seg] + t * 128;
-  valid = min(128, p.seg_len[seg] - t * 128);
+  // seg is 0 or 1: select rather than index, so the parameters stay in constant space
+  const int row0_s = seg ? p.seg_row0[1] : p.seg_row0[0];
+  const int len_s = seg ? p.seg_len[1] : p.seg_len[0];
+  row0 = row0_s + b * len_s + t * 128;
+  valid = min(128, (seg == p.nseg - 1 ? last_n : len_s) - t * 128);
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, A (bf16) read from TMEM.
@@ -145,8 +162,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   if (device_error_set()) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.y, b = blockIdx.z;
-  int n_kv = (p.seg_len[0] + 127) / 128;
-  if (p.nseg > 1) n_kv += (p.seg_len[1] + 127) / 128;
+  const int last_keys = attn_last_keys(p, b);
+  const int n_kv = p.nseg > 1 ? (p.seg_len[0] + 127) / 128 + (last_keys + 127) / 128 : (last_keys + 127) / 128;
   const int tile_a = 2 * blockIdx.x;
   const bool has_b = tile_a + 1 < p.q_tiles;  // CTA-uniform: the last CTA may hold one tile
 
@@ -187,8 +204,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const bool kq = warp == 8;
       if (kq) {
         int qa0, qav, qb0 = 0, qbv = 0;
-        attn_tile_rows(p, b, tile_a, qa0, qav);
-        if (has_b) attn_tile_rows(p, b, tile_a + 1, qb0, qbv);
+        attn_tile_rows(p, b, tile_a, attn_last_len(p), qa0, qav);
+        if (has_b) attn_tile_rows(p, b, tile_a + 1, attn_last_len(p), qb0, qbv);
         mbar_arrive_expect_tx(q_full, has_b ? 2 * kTile : kTile);
         tma_load_2d(smem + kQ0, &tm, q_full, colq, qa0);
         tma_load_2d(smem + kQ0 + kHalf, &tm, q_full, colq + 64, qa0);
@@ -207,7 +224,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const int bi = j & 1;
         const uint32_t r = uint32_t(j) >> 1;
         int kv0, kvn;
-        attn_tile_rows(p, b, j, kv0, kvn);
+        attn_tile_rows(p, b, j, last_keys, kv0, kvn);
         if (!mbar_wait(&emptyb[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) { ok = false; break; }
         mbar_arrive_expect_tx(&fullb[bi], kTile);
         tma_load_2d(smem + base + bi * kTile, &tm, &fullb[bi], col, kv0);
@@ -300,7 +317,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const int i = q * 32 + lane;  // query row in the tile == TMEM lane
     if (t == 0 || has_b) {
       int q_row0, q_valid;
-      attn_tile_rows(p, b, tile_a + t, q_row0, q_valid);
+      attn_tile_rows(p, b, tile_a + t, attn_last_len(p), q_row0, q_valid);
       const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
       const uint32_t s_addr = lane_addr + kColS + 128 * t;
       const uint32_t o_addr = lane_addr + kColO + 128 * t;
@@ -310,7 +327,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
         int kv0, kvn;
-        attn_tile_rows(p, b, j, kv0, kvn);
+        attn_tile_rows(p, b, j, last_keys, kv0, kvn);
         if (!mbar_wait(&s_full[t], uint32_t(j) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll

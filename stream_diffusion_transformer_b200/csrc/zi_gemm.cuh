@@ -22,10 +22,14 @@ namespace zi {
 // in one sequence's position table.  Rows [0, n_a) hold segment A (len_a rows
 // per batch element), rows [n_a, ...) hold segment B (len_b rows per element);
 // in a sequence, segment A occupies positions [0, len_a) and B [len_a, len_a + len_b).
+// tab_stride: rows of the position (RoPE) table per batch element; 0 when the
+// elements share one table, len_a + len_b when each element has its own.
 struct RowMap {
   int n_a, len_a, len_b;
+  int tab_stride;
   ZI_DEV int batch(int r) const { return r < n_a ? r / len_a : (r - n_a) / len_b; }
   ZI_DEV int pos(int r) const { return r < n_a ? r % len_a : len_a + (r - n_a) % len_b; }
+  ZI_DEV int tab(int r) const { return (tab_stride ? batch(r) * tab_stride : 0) + pos(r); }
 };
 
 enum EpiKind : int {
@@ -128,7 +132,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
       return;
     }
     const uint16_t* g = region == 0 ? ep.g_q : ep.g_k;
-    const int p = row_ok ? ep.map.pos(row + ep.row_off) : 0;
+    const int p = row_ok ? ep.map.tab(row + ep.row_off) : 0;
     const float2* rp = ep.rope + size_t(p) * 64;
 #pragma unroll 1
     for (int hh = 0; hh < width / 128; ++hh) {

@@ -205,6 +205,55 @@ __global__ void positions_kernel(int s_txt, int grid_h, int grid_w, int* __restr
   pos[3 * t + 2] = c;
 }
 
+// Positions of a padded batch, one sequence per element b: [image; s_txt text
+// rows], element b holding len[b] valid text tokens.  Image token (r, c) ->
+// (len[b] + 1, r, c); text row j (valid or pad) -> (j + 1, 0, 0).  With the pad
+// keys masked, this gives each element the positions of its unpadded sequence.
+// pos int32 [batch][grid_h*grid_w + s_txt][3].
+__global__ void positions_varlen_kernel(int s_txt, int grid_h, int grid_w, const int* __restrict__ len, int batch,
+                                        int* __restrict__ pos) {
+  const int n_img = grid_h * grid_w;
+  const int S = n_img + s_txt;
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<long long>(S) * batch) return;
+  const int b = int(t / S), i = int(t % S);
+  int a0, a1, a2;
+  if (i < n_img) {
+    a0 = len[b] + 1;
+    a1 = i / grid_w;
+    a2 = i % grid_w;
+  } else {
+    a0 = i - n_img + 1;
+    a1 = 0;
+    a2 = 0;
+  }
+  pos[3 * t + 0] = a0;
+  pos[3 * t + 1] = a1;
+  pos[3 * t + 2] = a2;
+}
+
+// Up to kLenChunk per-element text lengths carried by value into device memory
+// (no host-to-device copy, so the forward stays capturable in a CUDA graph).
+constexpr int kLenChunk = 64;
+struct LenChunk {
+  int n;
+  int v[kLenChunk];
+};
+
+__global__ void store_lengths_kernel(LenChunk c, int* __restrict__ out) {
+  if (int(threadIdx.x) < c.n) out[threadIdx.x] = c.v[threadIdx.x];
+}
+
+// Text rows j >= len[b] of element b take the cap_pad_token embedding (bf16 [D]).
+// x_txt fp32 [batch][s_txt][D]; grid (s_txt, batch), 256 threads.
+__global__ void text_pad_kernel(float* __restrict__ x_txt, int s_txt, int D, const int* __restrict__ len,
+                                const uint16_t* __restrict__ pad) {
+  const int j = blockIdx.x, b = blockIdx.y;
+  if (j < len[b]) return;
+  float* row = x_txt + (static_cast<size_t>(b) * s_txt + j) * D;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) row[i] = bf16_to_f32(pad[i]);
+}
+
 // (cos, sin) of pos[axis] * theta^(-2j/d_axis) for every token and rotation
 // pair; pairs [0, a0/2) use axis 0, the next a1/2 axis 1, the last a2/2 axis 2.
 // Angles are formed in fp64 and rounded to fp32 once.

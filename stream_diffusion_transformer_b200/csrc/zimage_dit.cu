@@ -184,14 +184,14 @@ EpiParams epi_plain(void* out, int ldo) {
   memset(&e, 0, sizeof(e));
   e.out = out;
   e.ldo = ldo;
-  e.map = RowMap{1, 1, 1};
+  e.map = RowMap{1, 1, 1, 0};
   return e;
 }
 
 // ---------------------------------------------------------------- attention
 
 int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out, int dim, int heads, int batch,
-                  int nseg, const int* row0, const int* len, cudaStream_t st) {
+                  int nseg, const int* row0, const int* len, const int* kv_len, cudaStream_t st) {
   CUtensorMap tm;
   ZI_TRY(make_map(&tm, qkv, uint64_t(3 * dim), uint64_t(qkv_rows), uint64_t(3 * dim) * 2, 64, 128));
   ZI_TRY(ensure_smem(dev, BIT_ATTN, attention_kernel, int(attn::kSmemBytes)));
@@ -209,6 +209,7 @@ int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out
   }
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(128.0));
   p.q_tiles = qt;
+  p.kv_len = kv_len;
   dim3 grid((qt + 1) / 2, heads, batch);  // two query tiles per CTA
   prof_pre(st);
   attention_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(tm, p);
@@ -239,7 +240,7 @@ constexpr size_t kAlign = 1024;
 inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-  size_t mod, c, silu, hid, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
+  size_t mod, c, silu, hid, lens, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
 };
 
 Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int mod_cols) {
@@ -254,8 +255,11 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.c = o; o = up(o + (model ? size_t(batch) * 256 * 4 : 0));
   w.silu = o; o = up(o + (model ? size_t(batch) * 256 * 4 : 0));
   w.hid = o; o = up(o + (model ? size_t(batch) * size_t(cfg.t_mid) * 4 : 0));
-  w.pos = o; o = up(o + (model ? S * 3 * 4 : 0));
-  w.rope = o; o = up(o + S * pairs * 8);
+  // a model forward may give every batch element its own positions (text lengths)
+  const size_t tab_rows = model ? rows : S;
+  w.lens = o; o = up(o + (model ? size_t(batch) * 4 : 0));
+  w.pos = o; o = up(o + (model ? tab_rows * 3 * 4 : 0));
+  w.rope = o; o = up(o + tab_rows * pairs * 8);
   w.x = o; o = up(o + (model ? rows * D * 4 : 0));
   w.h = o; o = up(o + rows * D * 2);
   w.qkv = o; o = up(o + rows * 3 * D * 2);
@@ -327,6 +331,7 @@ struct BlockCtx {
   int mod_ld;
   int nseg;
   int seg_row0[2], seg_len[2];  // local rows
+  const int* kv_len;  // [batch] keys of the last segment (valid text tokens), or null = all
 };
 
 int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
@@ -343,7 +348,8 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   eq.row_off = b.row_off;
   eq.map = b.map;
   ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st)));
-  ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len, st));
+  ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len,
+                       b.kv_len, st));
   ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D, epi_plain(b.o, D), st)));
   PostParams pa;
   memset(&pa, 0, sizeof(pa));
@@ -572,7 +578,19 @@ int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
   const int row0[1] = {0}, len[1] = {seq};
-  return run_attention(dev, d_qkv, batch * seq, d_out, heads * 128, heads, batch, 1, row0, len,
+  return run_attention(dev, d_qkv, batch * seq, d_out, heads * 128, heads, batch, 1, row0, len, nullptr,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int zi_attention_varlen(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads,
+                        const int32_t* d_kv_len, zi_stream_t stream) {
+  if (!d_qkv || !d_out || !d_kv_len || batch <= 0 || seq <= 0 || heads <= 0) return ZI_ERR_ARG;
+  if (!aligned16(d_qkv) || !aligned16(d_out) || (reinterpret_cast<uintptr_t>(d_kv_len) & 3u)) return ZI_ERR_ALIGN;
+  if (heads > 65535 || batch > 65535) return ZI_ERR_SHAPE;
+  DevInfo* dev;
+  ZI_TRY(current_device(&dev));
+  const int row0[1] = {0}, len[1] = {seq};
+  return run_attention(dev, d_qkv, batch * seq, d_out, heads * 128, heads, batch, 1, row0, len, d_kv_len,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -618,7 +636,7 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.rows = rows;
   b.row_off = 0;
   b.batch = batch;
-  b.map = RowMap{rows, seq, 1};
+  b.map = RowMap{rows, seq, 1, 0};
   b.x_in = const_cast<float*>(d_x_in);
   b.x_out = d_x_out;
   b.h = reinterpret_cast<uint16_t*>(ws + L.h);
@@ -634,6 +652,7 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.seg_len[0] = seq;
   b.seg_row0[1] = 0;
   b.seg_len[1] = 1;
+  b.kv_len = nullptr;
   ZI_TRY(run_rms_mod<float>(d_x_in, rows, D, w->g_attn1, b.mod, b.mod_ld, b.map, 0, cfg->norm_eps, b.h, st));
   const NextNormSpec none{NEXT_NONE, nullptr, nullptr, 0};
   return run_block(b, none, st);
@@ -657,11 +676,16 @@ int zi_block_forward_noalloc(const zi_config* cfg, const zi_block_weights* w, co
 
 namespace {
 int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
-                       const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, float* d_trace,
-                       void* d_ws, size_t ws_bytes, zi_stream_t stream) {
+                       const int32_t* h_txt_len, const float* d_latent, const float* d_t, const uint16_t* d_txt,
+                       float* d_out, float* d_trace, void* d_ws, size_t ws_bytes, zi_stream_t stream) {
   ZI_TRY(check_cfg(cfg));
   if (!w || !d_latent || !d_t || !d_txt || !d_out || batch <= 0 || lat_h <= 0 || lat_w <= 0 || s_txt <= 0)
     return ZI_ERR_ARG;
+  if (h_txt_len) {
+    if (!w->cap_pad) return ZI_ERR_ARG;
+    for (int b = 0; b < batch; ++b)
+      if (h_txt_len[b] < 1 || h_txt_len[b] > s_txt) return ZI_ERR_ARG;
+  }
   if (lat_h % 2 || lat_w % 2) return ZI_ERR_SHAPE;
   if (batch > 65535) return ZI_ERR_SHAPE;
   const void* top[] = {w->x_emb_w, w->x_emb_b, w->cap_norm, w->cap_w, w->cap_b, w->t_w1, w->t_b1, w->t_w2,
@@ -707,7 +731,8 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   uint16_t* u = reinterpret_cast<uint16_t*>(ws + L.u);
   uint16_t* tok = reinterpret_cast<uint16_t*>(ws + L.tok);
   uint16_t* capn = reinterpret_cast<uint16_t*>(ws + L.capn);
-  const RowMap map{rows_img, s_img, s_txt};
+  int* lens = h_txt_len ? reinterpret_cast<int*>(ws + L.lens) : nullptr;
+  const RowMap map{rows_img, s_img, s_txt, h_txt_len ? S : 0};
   const float eps = cfg->norm_eps;
   int traced = 0;
   auto trace = [&]() -> int {
@@ -756,11 +781,29 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   auto mod_of_main = [&](int i) { return mod + size_t(cfg->n_noise + i) * 4 * D; };
   const float* final_scale = mod + size_t(n_mod) * 4 * D;
 
-  // positions and RoPE table of one sequence [image; text]
-  prof_pre(st);
-  positions_kernel<<<(S + 255) / 256, 256, 0, st>>>(s_txt, gh, gw, pos);
-  ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
-  ZI_TRY(run_rope(*cfg, pos, S, rope, st));
+  // positions and RoPE table: one sequence [image; text] shared by the batch, or,
+  // with text lengths, one per element (its image positions follow its length)
+  if (!h_txt_len) {
+    prof_pre(st);
+    positions_kernel<<<(S + 255) / 256, 256, 0, st>>>(s_txt, gh, gw, pos);
+    ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
+    ZI_TRY(run_rope(*cfg, pos, S, rope, st));
+  } else {
+    for (int b0 = 0; b0 < batch; b0 += kLenChunk) {
+      LenChunk ch;
+      memset(&ch, 0, sizeof(ch));
+      ch.n = batch - b0 < kLenChunk ? batch - b0 : kLenChunk;
+      for (int i = 0; i < ch.n; ++i) ch.v[i] = h_txt_len[b0 + i];
+      prof_pre(st);
+      store_lengths_kernel<<<1, kLenChunk, 0, st>>>(ch, lens + b0);
+      ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
+    }
+    const long long n = static_cast<long long>(rows);
+    prof_pre(st);
+    positions_varlen_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(s_txt, gh, gw, lens, batch, pos);
+    ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
+    ZI_TRY(run_rope(*cfg, pos, rows, rope, st));
+  }
 
   // embedders: image rows [0, rows_img), text rows [rows_img, rows)
   {
@@ -776,6 +819,11 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     EpiParams ec = epi_plain(x + size_t(rows_img) * D, D);
     ec.bias = w->cap_b;
     ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, capn, w->cap_w, rows_txt, D, cfg->cap_dim, ec, st)));
+    if (h_txt_len) {
+      prof_pre(st);
+      text_pad_kernel<<<dim3(s_txt, batch), 256, 0, st>>>(x + size_t(rows_img) * D, s_txt, D, lens, w->cap_pad);
+      ZI_TRY(launched(ZI_KERNEL_TEXT_PAD, st));
+    }
   }
 
   BlockCtx base;
@@ -785,6 +833,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   base.map = map;
   base.rope = rope;
   base.mod_ld = mod_ld;
+  base.kv_len = lens;
 
   auto segment_ctx = [&](int row_off, int nrows, int seglen) {
     BlockCtx b = base;
@@ -806,9 +855,10 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   };
   const NextNormSpec to_main0{NEXT_RMS, w->main[0].g_attn1, mod_of_main(0), 0};
 
-  // noise refiners on the image rows
+  // noise refiners on the image rows (all keys are image tokens: no key mask)
   {
     BlockCtx b = segment_ctx(0, rows_img, s_img);
+    b.kv_len = nullptr;
     if (cfg->n_noise > 0) {
       ZI_TRY(run_rms_mod<float>(b.x_in, rows_img, D, w->noise[0].g_attn1, mod_of_noise(0), mod_ld, map, 0, eps,
                                 b.h, st));
@@ -881,8 +931,16 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
 int zi_model_forward(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w, int s_txt,
                      const float* d_latent, const float* d_t, const uint16_t* d_txt, float* d_out, void* d_ws,
                      size_t ws_bytes, zi_stream_t stream) {
-  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, d_latent, d_t, d_txt, d_out, nullptr, d_ws, ws_bytes,
-                            stream);
+  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, nullptr, d_latent, d_t, d_txt, d_out, nullptr, d_ws,
+                            ws_bytes, stream);
+}
+
+int zi_model_forward_varlen(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w,
+                            int s_txt, const int32_t* h_txt_len, const float* d_latent, const float* d_t,
+                            const uint16_t* d_txt, float* d_out, void* d_ws, size_t ws_bytes, zi_stream_t stream) {
+  if (!h_txt_len) return ZI_ERR_ARG;
+  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, h_txt_len, d_latent, d_t, d_txt, d_out, nullptr, d_ws,
+                            ws_bytes, stream);
 }
 
 int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* w, int batch, int lat_h, int lat_w,
@@ -890,8 +948,8 @@ int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* w, int 
                            float* d_trace, void* d_ws, size_t ws_bytes, zi_stream_t stream) {
   if (!d_trace) return ZI_ERR_ARG;
   if (!aligned16(d_trace)) return ZI_ERR_ALIGN;
-  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, d_latent, d_t, d_txt, d_out, d_trace, d_ws, ws_bytes,
-                            stream);
+  return model_forward_impl(cfg, w, batch, lat_h, lat_w, s_txt, nullptr, d_latent, d_t, d_txt, d_out, d_trace, d_ws,
+                            ws_bytes, stream);
 }
 
 int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond, float guidance, double sigma,

@@ -62,6 +62,7 @@ TOP_KEYS = {
     "t_w2": "t_embedder.linear2.weight", "t_b2": "t_embedder.linear2.bias",
     "final_ada_w": "final_layer.adaLN_modulation.weight", "final_ada_b": "final_layer.adaLN_modulation.bias",
     "final_w": "final_layer.linear.weight", "final_b": "final_layer.linear.bias",
+    "cap_pad": "cap_pad_token",
 }
 
 
@@ -124,6 +125,7 @@ class DiT:
         self._main_arr = (abi.ZiBlockWeights * len(self.main))(*[b.struct for b in self.main])
         kw = {f: self.top[f].data_ptr() for f in abi.MODEL_FIELDS}
         self.weights = abi.ZiModelWeights(**kw)
+        self.weights.cap_pad = self.top["cap_pad"].data_ptr()
         self.weights.noise = ctypes.cast(self._noise_arr, ctypes.POINTER(abi.ZiBlockWeights))
         self.weights.ctx = ctypes.cast(self._ctx_arr, ctypes.POINTER(abi.ZiBlockWeights))
         self.weights.main = ctypes.cast(self._main_arr, ctypes.POINTER(abi.ZiBlockWeights))
@@ -141,12 +143,16 @@ class DiT:
         return self._ws[key]
 
     def denoise(self, latent: torch.Tensor, txt: torch.Tensor, n_steps: int = 8, shift: float = 3.0,
-                guidance: Optional[float] = None, txt_uncond: Optional[torch.Tensor] = None) -> torch.Tensor:
+                guidance: Optional[float] = None, txt_uncond: Optional[torch.Tensor] = None,
+                txt_len: Optional[Sequence[int]] = None,
+                txt_uncond_len: Optional[Sequence[int]] = None) -> torch.Tensor:
         """FlowMatch-Euler loop (z-image-turbo-mnn "Scheduler"): n_steps forwards at
         t = 1 - sigma'_i, each followed by zi_euler_step with sigma'_i -> sigma'_{i+1};
         with guidance and txt_uncond, the conditional and unconditional branches run
-        as one batch-2 forward and are combined y_u + g (y_c - y_u).  Returns the
-        final latent (a new tensor; `latent` is left unchanged)."""
+        as one batch-2 forward and are combined y_u + g (y_c - y_u).  txt_len /
+        txt_uncond_len give the real lengths of padded prompts (see forward); the
+        two branches' texts are padded to one length.  Returns the final latent (a
+        new tensor; `latent` is left unchanged)."""
         sig = abi.sigmas(n_steps, shift)
         x = latent.clone()
         B = x.shape[0]
@@ -154,14 +160,25 @@ class DiT:
         out = torch.empty((2 * B,) + tuple(x.shape[1:]) if cfg_mode else x.shape, dtype=torch.float32,
                           device=x.device)
         tt = torch.empty(2 * B if cfg_mode else B, dtype=torch.float32, device=x.device)
-        txt_all = torch.cat([txt, txt_uncond], 0) if cfg_mode else txt
+        lens = None if txt_len is None else list(txt_len)
+        if cfg_mode:
+            L = max(txt.shape[1], txt_uncond.shape[1])
+            if txt.shape[1] != txt_uncond.shape[1] or txt_len is not None or txt_uncond_len is not None:
+                lc = list(txt_len) if txt_len is not None else [txt.shape[1]] * B
+                lu = list(txt_uncond_len) if txt_uncond_len is not None else [txt_uncond.shape[1]] * B
+                lens = lc + lu
+            txt_all = torch.zeros((2 * B, L, txt.shape[2]), dtype=txt.dtype, device=txt.device)
+            txt_all[:B, :txt.shape[1]].copy_(txt)
+            txt_all[B:, :txt_uncond.shape[1]].copy_(txt_uncond)
+        else:
+            txt_all = txt
         x_in = torch.empty((2 * B,) + tuple(x.shape[1:]), dtype=torch.float32, device=x.device) if cfg_mode else x
         for i in range(n_steps):
             tt.fill_(1.0 - sig[i])
             if cfg_mode:
                 x_in[:B].copy_(x)
                 x_in[B:].copy_(x)
-            self.forward(x_in, tt, txt_all, out)
+            self.forward(x_in, tt, txt_all, out, txt_len=lens)
             if cfg_mode:
                 abi.call("zi_euler_step", _p(x), _p(out[:B]), _p(out[B:]), float(guidance), sig[i], sig[i + 1],
                          x.numel(), _stream())
@@ -170,8 +187,12 @@ class DiT:
         return x
 
     def forward(self, latent: torch.Tensor, t: torch.Tensor, txt: torch.Tensor,
-                out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-        """latent fp32 [B, C, H/8, W/8], t fp32 [B] (1 = clean), txt bf16 [B, L, cap_dim] -> raw output."""
+                out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                txt_len: Optional[Sequence[int]] = None) -> torch.Tensor:
+        """latent fp32 [B, C, H/8, W/8], t fp32 [B] (1 = clean), txt bf16 [B, L, cap_dim] -> raw output.
+
+        txt_len (host ints, one per element, each in [1, L]): element b's prompt is
+        its first txt_len[b] text rows, the rest padding (zi_model_forward_varlen)."""
         B, C, Hl, Wl = latent.shape
         L = txt.shape[1]
         assert latent.dtype == torch.float32 and t.dtype == torch.float32 and txt.dtype == torch.bfloat16
@@ -179,8 +200,13 @@ class DiT:
         if out is None:
             out = torch.empty_like(latent)
         ws = self.workspace(B, Hl, Wl, L)
-        abi.call("zi_model_forward", ctypes.byref(self.cfg), ctypes.byref(self.weights), B, Hl, Wl, L,
-                 _p(latent), _p(t), _p(txt), _p(out), _p(ws), ws.numel(), _stream(stream))
+        if txt_len is None:
+            abi.call("zi_model_forward", ctypes.byref(self.cfg), ctypes.byref(self.weights), B, Hl, Wl, L,
+                     _p(latent), _p(t), _p(txt), _p(out), _p(ws), ws.numel(), _stream(stream))
+        else:
+            lens = (ctypes.c_int32 * B)(*[int(v) for v in txt_len])
+            abi.call("zi_model_forward_varlen", ctypes.byref(self.cfg), ctypes.byref(self.weights), B, Hl, Wl, L,
+                     lens, _p(latent), _p(t), _p(txt), _p(out), _p(ws), ws.numel(), _stream(stream))
         return out
 
 
@@ -240,10 +266,14 @@ def gemm(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None) -
 
 
 def attention(qkv: torch.Tensor, batch: int, seq: int, heads: int,
-              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+              out: Optional[torch.Tensor] = None, kv_len: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """kv_len: device int32 [batch] of valid keys per element (the rest masked), or None."""
     if out is None:
         out = torch.empty((batch * seq, heads * 128), dtype=torch.bfloat16, device=qkv.device)
-    abi.call("zi_attention", _p(qkv), _p(out), batch, seq, heads, _stream())
+    if kv_len is None:
+        abi.call("zi_attention", _p(qkv), _p(out), batch, seq, heads, _stream())
+    else:
+        abi.call("zi_attention_varlen", _p(qkv), _p(out), batch, seq, heads, _p(kv_len), _stream())
     return out
 
 

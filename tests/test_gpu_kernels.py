@@ -123,6 +123,27 @@ def test_attention(M, batch, seq, heads):
         assert_parity(got[b], want, rel=1e-2, cos=0.9999, what=f"attention b={b}")
 
 
+@pytest.mark.parametrize("seq,kv_len", [(300, [1, 77, 300, 129]), (256, [128, 255, 256, 2])])
+def test_attention_key_mask(M, seq, kv_len):
+    """Per-element key counts (padding masked as keys): one key, a count inside a tile,
+    exactly a tile boundary, all keys, one past a boundary; every query row checked."""
+    abi, model = M
+    heads, batch = 2, len(kv_len)
+    D = heads * 128
+    qkv = zi.make_matrix((batch * seq, 3 * D), 4, seq + 7)
+    lens = torch.tensor(kv_len, dtype=torch.int32, device="cuda")
+    out = model.attention(dev_bits(qkv), batch, seq, heads, kv_len=lens)
+    torch.cuda.synchronize()
+    got = host_f64(out).reshape(batch, seq, heads, 128)
+    x = bits_f64(qkv).reshape(batch, seq, 3, heads, 128)
+    for b in range(batch):
+        valid = np.arange(seq) < kv_len[b]
+        want = ref.attention(x[b, :, 0], x[b, :, 1], x[b, :, 2], key_valid=valid)
+        assert_parity(got[b], want, rel=1e-2, cos=0.9999, what=f"masked attention b={b} keys={kv_len[b]}")
+        if kv_len[b] == 1:  # a single key: every query's output is that key's value row
+            np.testing.assert_allclose(got[b], np.broadcast_to(x[b, 0, 2], got[b].shape), rtol=0, atol=0)
+
+
 def test_attention_sharp_scores(M):
     """Large logits: the running max moves by far more than 2^8 between key tiles."""
     abi, model = M

@@ -97,3 +97,60 @@ def test_cfg_loop_batch2():
     got, want, x0 = _denoise_case(zi.TINY_R, 8, 16, 4, seed=4, guidance=4.0)
     assert_parity(got, want, rel=3e-2, cos=0.995, what="CFG loop final latent")
     assert_parity(got - x0, want - x0, rel=3e-2, cos=0.995, what="CFG loop latent change")
+
+
+def test_variable_length_text_batch():
+    """Prompts of 20 and 7 tokens padded to 20 (cap_pad_token rows, masked as keys):
+    each element against the oracle's padded batch, and element 1 against the
+    oracle run on its unpadded 7-token prompt alone."""
+    from stream_diffusion_transformer_b200 import model
+    d = zi.TINY_R
+    bits = zi.make_weights(d, seed=5)
+    dit = model.DiT(model.make_config(d), lambda keys: {k: bits[k] for k in keys})
+    lat = zi.make_latent(d, 2, 10, 12, seed=5)
+    txt = zi.make_text(d, 2, 20, seed=5)
+    txt[1, 7:] = 0x7F80  # +inf bits in the padding rows: they must not reach the output
+    tt = np.array([0.35, 0.6], dtype=np.float32)
+    lens = [20, 7]
+    out = dit.forward(torch.from_numpy(lat).cuda(), torch.from_numpy(tt).cuda(),
+                      torch.from_numpy(txt.view(np.int16)).cuda().view(torch.bfloat16), txt_len=lens)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    W = ref.Weights(bits)
+    tf = zi.bf16_bits_to_f32(txt).astype(np.float64)
+    tf[1, 7:] = 0.0
+    want = ref.model_forward(lat.astype(np.float64), tt.astype(np.float64), tf, W, d, txt_len=np.array(lens))
+    for b in range(2):
+        assert_parity(got[b], want[b], rel=3e-2, cos=0.995, what=f"varlen b={b} len={lens[b]}")
+    alone = ref.model_forward(lat[1:].astype(np.float64), tt[1:].astype(np.float64), tf[1:, :7], W, d)
+    assert_parity(got[1:], alone, rel=3e-2, cos=0.995, what="varlen b=1 vs unpadded alone")
+
+
+def test_variable_length_cfg_loop_full_width():
+    """CFG loop at full width (1 + 1 + 2 blocks, 256 image tokens): a 96-token prompt and
+    a 9-token negative prompt padded to one 96-row batch-2 forward per step, against the
+    oracle's loop that runs each branch on its own unpadded text."""
+    from oracle import scheduler_ref as sch
+    from stream_diffusion_transformer_b200 import model
+    d = dataclasses.replace(zi.FULL, n_noise=1, n_ctx=1, n_main=2)
+    bits = zi.make_weights(d, seed=6, threads=8)
+    dit = model.DiT(model.make_config(d), lambda keys: {k: bits[k] for k in keys})
+    lat = zi.make_latent(d, 1, 32, 32, seed=6)
+    txt = zi.make_text(d, 1, 96, seed=6)
+    txt_u = zi.make_text(d, 1, 9, seed=6, uncond=True)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+    got = dit.denoise(torch.from_numpy(lat).cuda(), dev(txt), n_steps=3, shift=3.0, guidance=4.0,
+                      txt_uncond=dev(txt_u))
+    torch.cuda.synchronize()
+    W = ref.Weights(bits)
+    tc = zi.bf16_bits_to_f32(txt).astype(np.float64)
+    tu = zi.bf16_bits_to_f32(txt_u).astype(np.float64)
+
+    def model_fn(x, t, uncond):
+        return ref.model_forward(x, t, tu if uncond else tc, W, d)
+
+    x0 = lat.astype(np.float64)
+    want = sch.denoise(x0, model_fn, 3, 3.0, 4.0)
+    g = got.cpu().numpy().astype(np.float64)
+    assert_parity(g, want, rel=3e-2, cos=0.995, what="varlen CFG loop final latent")
+    assert_parity(g - x0, want - x0, rel=3e-2, cos=0.995, what="varlen CFG loop latent change")

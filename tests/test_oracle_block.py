@@ -218,3 +218,38 @@ def test_trace_records_every_block():
     tr = []
     ref.model_forward(lat, np.array([0.5]), txt, W, d, trace=tr)
     assert [t.shape for t in tr] == [(4, 256), (3, 256), (7, 256)]
+
+
+def test_padding_is_invisible_with_the_key_mask():
+    """Variable-length text: element 1 padded from 3 to 7 text tokens (pad rows hold
+    cap_pad_token, masked as keys) gives the output of running it unpadded."""
+    d = zi.TINY_R
+    W = ref.Weights(_weights(d, 8))
+    lat = zi.make_latent(d, 2, 4, 6, seed=8).astype(np.float64)
+    txt = zi.bf16_bits_to_f32(zi.make_text(d, 2, 7, seed=8)).astype(np.float64)
+    t = np.array([0.4, 0.7])
+    lens = np.array([7, 3])
+    padded = ref.model_forward(lat, t, txt, W, d, txt_len=lens)
+    full0 = ref.model_forward(lat[:1], t[:1], txt[:1], W, d)
+    short1 = ref.model_forward(lat[1:], t[1:], txt[1:, :3], W, d)
+    np.testing.assert_allclose(padded[:1], full0, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(padded[1:], short1, rtol=1e-10, atol=1e-12)
+
+
+def test_pad_token_value_and_pad_features_do_not_leak():
+    d = zi.TINY_R
+    bits = _weights(d, 9)
+    lat = zi.make_latent(d, 1, 4, 4, seed=9).astype(np.float64)
+    txt = zi.bf16_bits_to_f32(zi.make_text(d, 1, 6, seed=9)).astype(np.float64)
+    t = np.array([0.5])
+    lens = np.array([2])
+    base = ref.model_forward(lat, t, txt, ref.Weights(bits), d, txt_len=lens)
+    txt2 = txt.copy()
+    txt2[:, 2:] *= -3.0
+    b2 = dict(bits)
+    b2["cap_pad_token"] = zi.f32_to_bf16_bits(zi.bf16_bits_to_f32(bits["cap_pad_token"]) * np.float32(5.0))
+    np.testing.assert_allclose(ref.model_forward(lat, t, txt2, ref.Weights(b2), d, txt_len=lens), base,
+                               rtol=1e-10, atol=1e-12)
+    # without the key mask the pads would change the image tokens
+    unmasked = ref.model_forward(lat, t, txt, ref.Weights(bits), d)
+    assert np.abs(unmasked - base).max() > 1e-4
