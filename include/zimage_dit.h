@@ -325,7 +325,8 @@ enum zi_kernel_kind {
   ZI_KERNEL_GEMM_FINAL = 14,    /* final linear + unpatchify */
   ZI_KERNEL_EULER = 15,         /* Euler / CFG step */
   ZI_KERNEL_GEMM = 16,          /* zi_gemm_bf16 */
-  ZI_KERNEL_TEXT_PAD = 17       /* cap_pad_token into padded text rows */
+  ZI_KERNEL_TEXT_PAD = 17,      /* cap_pad_token into padded text rows */
+  ZI_KERNEL_SPLIT_CLEAR = 18    /* zero the GEMM split-tail counters (once per forward) */
 };
 
 /* Start recording launch timings on this host thread: from the next kernel the

@@ -162,7 +162,7 @@ KERNEL_NAMES = {
     1: "gemm_qkv_qknorm_rope", 2: "attention", 3: "gemm_out_proj", 4: "gemm_ffn_up_swiglu",
     5: "gemm_ffn_down", 6: "post_norm_residual", 7: "pre_norm", 8: "adaln_gemv", 9: "timestep_mlp",
     10: "rope_table", 11: "positions", 12: "patchify", 13: "gemm_embed", 14: "gemm_final_unpatchify",
-    15: "euler", 16: "gemm", 17: "text_pad",
+    15: "euler", 16: "gemm", 17: "text_pad", 18: "split_clear",
 }
 
 

@@ -208,38 +208,45 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
 }
 
 // Work schedule.  T output tiles of 128 x BN run on G persistent CTAs, tile t
-// on CTA t % G.  When T % G leaves a last wave of R < G tiles, and f R <= G for
-// a split factor f in {2, 4} the epilogue allows, those R tiles are cut along N
-// into f sub-tiles of BN / f columns each, one per CTA: the ragged wave then
-// costs 1/f of a tile's time instead of a whole one, with no reduction across
-// CTAs.
+// on CTA t % G.  When T % G leaves a last wave of R < G tiles, those R tiles are
+// cut along K into s pieces (s R <= G, s <= kMaxSplit, at least kMinSplitKb
+// k-blocks each), one piece per CTA, so the ragged wave costs about 1/s of a
+// tile's time.  (Cutting along N instead would not help: a tcgen05.mma with
+// A and B in shared memory takes about as long at N = 64 or 128 as at 256.)
+// Every piece stores its fp32 partial tile in its own slot and bumps the tile's
+// counter; the piece that completes the count adds the partials in slot order
+// (the same order whichever piece finishes, so results are deterministic) and
+// runs the fused epilogue.  No CTA waits for another.
+constexpr int kMaxSplit = 4;
+constexpr int kMinSplitKb = 4;
+constexpr int kSplitSlots = 160;  // partial slots (>= G); counters likewise
+
 struct TailSched {
   int grid;        // G
   int dp_tiles;    // tiles [0, dp_tiles) run whole, walked with stride G
-  int tail_f;      // sub-tiles per tail tile (1 = no tail)
-  int tail_items;  // CTAs [0, tail_items) each run one sub-tile of tile dp_tiles + c / tail_f
+  int tail_s;      // K pieces per tail tile (1 = no tail)
+  int tail_items;  // CTAs [0, tail_items) each run piece c % s of tile dp_tiles + c / s
+  int kb;          // k-blocks per tile
 };
 
-inline TailSched make_tail_sched(int tiles, int grid, int max_f) {
-  TailSched s{grid, tiles, 1, 0};
-  if (tiles <= grid) return s;
+inline TailSched make_tail_sched(int tiles, int grid, int kb, bool can_split) {
+  TailSched s{grid, tiles, 1, 0, kb};
   const int rounds = tiles / grid, rest = tiles - rounds * grid;
-  if (rest == 0) return s;
-  for (int f = max_f; f >= 2; f /= 2) {
-    if (f * rest <= grid) {
-      s.dp_tiles = rounds * grid;
-      s.tail_f = f;
-      s.tail_items = f * rest;
-      return s;
-    }
-  }
+  if (!can_split || rest == 0 || grid > kSplitSlots) return s;
+  int f = grid / rest;
+  if (f > kMaxSplit) f = kMaxSplit;
+  if (f > kb / kMinSplitKb) f = kb / kMinSplitKb;
+  if (f < 2) return s;
+  s.dp_tiles = rounds * grid;
+  s.tail_s = f;
+  s.tail_items = f * rest;
   return s;
 }
 
 struct WorkItem {
-  int tile;   // 128 x BN tile index (M fastest)
-  int col0;   // first column of the item inside the tile
-  int width;  // columns of the item (BN, or BN / tail_f for a tail sub-tile)
+  int tile;      // 128 x BN tile index (M fastest)
+  int kb0, kb1;  // k-block range of this item
+  int piece;     // -1: the whole tile; else the piece index of a split tail tile
 };
 
 // Walks one CTA's work items; every warp role walks the same sequence.
@@ -248,31 +255,39 @@ struct WorkWalker {
   int c, next_dp;
   bool tail_done;
   ZI_DEV WorkWalker(const TailSched& sched, int cta) : s(sched), c(cta), next_dp(cta), tail_done(false) {}
-  template <int BN>
   ZI_DEV bool next(WorkItem& w) {
     if (next_dp < s.dp_tiles) {
       w.tile = next_dp;
-      w.col0 = 0;
-      w.width = BN;
+      w.kb0 = 0;
+      w.kb1 = s.kb;
+      w.piece = -1;
       next_dp += s.grid;
       return true;
     }
     if (!tail_done && c < s.tail_items) {
       tail_done = true;
-      w.width = BN / s.tail_f;
-      w.tile = s.dp_tiles + c / s.tail_f;
-      w.col0 = (c % s.tail_f) * w.width;
+      w.tile = s.dp_tiles + c / s.tail_s;
+      w.piece = c % s.tail_s;
+      w.kb0 = w.piece * s.kb / s.tail_s;
+      w.kb1 = (w.piece + 1) * s.kb / s.tail_s;
       return true;
     }
     return false;
   }
 };
 
+// Scratch of the split tail: partial tiles [kSplitSlots][BN / 4][128] float4
+// (column-quad major, so a warp's 32 rows store 512 contiguous bytes) and one
+// counter per tail tile, zero on entry (each tile's finisher puts it back to zero).
+struct SplitScratch {
+  float4* partials;
+  int* counters;
+};
+
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
-    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmB64, int M, int N, int K, EpiParams ep,
-                        TailSched sched) {
+    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                        int N, int K, EpiParams ep, TailSched sched, SplitScratch sk) {
   using L = GemmSmem<BN, STAGES>;
   constexpr int BM = 128, BK = 64;
   extern __shared__ uint8_t smem_raw[];
@@ -282,8 +297,10 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ebar = drain + 1;  // the epilogue warps' own barrier (split tail)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
 
   if (device_error_set()) return;  // an earlier kernel timed out: leave everything untouched
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -298,13 +315,13 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(ebar, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    prefetch_tmap(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
@@ -316,7 +333,6 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_m = (M + BM - 1) / BM;
-  const int KB = K / BK;
   WorkItem wi;
 
   if (warp == 0) {
@@ -324,10 +340,10 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0;
       bool ok = true;
       WorkWalker walk(sched, blockIdx.x);
-      while (ok && walk.next<BN>(wi)) {
-        const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN + wi.col0;
-        const uint32_t bytes = L::kABytes + uint32_t(wi.width) * 128u;
-        for (int kb = 0; kb < KB; ++kb) {
+      while (ok && walk.next(wi)) {
+        const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
+        const uint32_t bytes = L::kStage;
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) {
             ok = false;
@@ -336,14 +352,7 @@ __global__ void __launch_bounds__(192, 1)
           uint8_t* sa = smem + s * L::kStage;
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(sa, &tmA, &full[s], kb * BK, m0);
-          if (wi.width == BN) {
-            tma_load_2d(sa + L::kABytes, &tmB, &full[s], kb * BK, n0);
-          } else {
-            // a tail sub-tile: its B rows in 64-row boxes, which land 8 KB apart in
-            // the same swizzled layout one box of `width` rows would produce
-            for (int r64 = 0; r64 < wi.width / 64; ++r64)
-              tma_load_2d(sa + L::kABytes + r64 * 8192, &tmB64, &full[s], kb * BK, n0 + r64 * 64);
-          }
+          tma_load_2d(sa + L::kABytes, &tmB, &full[s], kb * BK, n0);
           ++it;
         }
       }
@@ -363,8 +372,8 @@ __global__ void __launch_bounds__(192, 1)
       int local = 0;
       bool ok = true;
       WorkWalker walk(sched, blockIdx.x);
-      while (ok && walk.next<BN>(wi)) {
-        const uint32_t idesc = idesc_bf16_f32(128, wi.width, false, false);
+      const uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      while (ok && walk.next(wi)) {
         const int acc = local & 1;
         const uint32_t u = uint32_t(local) >> 1;
         ++local;
@@ -374,7 +383,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&full[s], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
             ok = false;
@@ -386,7 +395,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             tc_mma(d, smem_desc_sw128(a_addr + k * 32, 16), smem_desc_sw128(b_addr + k * 32, 16), idesc,
-                   (kb | k) != 0 ? 1u : 0u);
+                   (kb != wi.kb0 || k != 0) ? 1u : 0u);
           }
           tc_commit(&empty[s]);
           ++it;
@@ -404,17 +413,90 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;  // this warp's TMEM lane quarter
     const int row_in_tile = q * 32 + lane;
     int local = 0;
+    uint32_t ephase = 0;
+    auto epi_sync = [&]() -> bool {  // the 128 epilogue threads meet (bounded wait)
+      mbar_arrive(ebar);
+      const bool r = mbar_wait(ebar, ephase, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE);
+      ephase ^= 1u;
+      return r;
+    };
     WorkWalker walk(sched, blockIdx.x);
-    while (walk.next<BN>(wi)) {
+    while (walk.next(wi)) {
       const int acc = local & 1;
       const uint32_t u = uint32_t(local) >> 1;
       ++local;
       if (!mbar_wait(&tfull[acc], u & 1u, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN + wi.col0;
+      const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
       const int row = m0 + row_in_tile;
       const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-      gemm_epilogue<EPI, BN>(tb, row, row < M, n0, wi.width, ep);
+      bool finish = true;
+      if (wi.piece >= 0) {
+        // A piece of a split tile: publish the partial, then finish only if last.
+        const int slot0 = blockIdx.x - wi.piece;  // slot of piece 0 of this tile
+        float4* mine = sk.partials + size_t(blockIdx.x) * (32 * BN) + row_in_tile;
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(tb + c * 32, v);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            __stcg(mine + size_t(c * 8 + k) * 128,
+                   make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                               __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+        }
+        __threadfence();
+        if (!epi_sync()) break;
+        if (threadIdx.x == 64) {
+          const int t = wi.tile - sched.dp_tiles;
+          const int old = atomicAdd(&sk.counters[t], 1);
+          const bool last = old == sched.tail_s - 1;
+          if (last) sk.counters[t] = 0;  // ready for the next launch
+          *last_flag = last ? 1 : 0;
+        }
+        if (!epi_sync()) break;
+        finish = *last_flag != 0;
+        if (finish) {
+          __threadfence();
+          for (int c = 0; c < BN / 32; ++c) {
+            // Every other piece's 32 columns are loaded before any is used, so up to
+            // (kMaxSplit - 1) x 8 loads are in flight instead of one at a time.
+            float4 pp[kMaxSplit][8];
+#pragma unroll
+            for (int j = 0; j < kMaxSplit; ++j) {
+              const bool need = j < sched.tail_s && j != wi.piece;
+              const float4* src = sk.partials + size_t(slot0 + j) * (32 * BN) + size_t(c * 8) * 128 + row_in_tile;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) pp[j][k] = need ? __ldcg(src + size_t(k) * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            uint32_t v[32];
+            tmem_ld32_sync(tb + c * 32, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 own = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                             __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+              // sum in piece order 0, 1, ..., s - 1 whichever piece finishes
+              float4 tot = wi.piece == 0 ? own : pp[0][k];
+#pragma unroll
+              for (int j = 1; j < kMaxSplit; ++j) {
+                if (j < sched.tail_s) {
+                  const float4 pj = j == wi.piece ? own : pp[j][k];
+                  tot.x += pj.x;
+                  tot.y += pj.y;
+                  tot.z += pj.z;
+                  tot.w += pj.w;
+                }
+              }
+              v[4 * k] = __float_as_uint(tot.x);
+              v[4 * k + 1] = __float_as_uint(tot.y);
+              v[4 * k + 2] = __float_as_uint(tot.z);
+              v[4 * k + 3] = __float_as_uint(tot.w);
+            }
+            tmem_st32(tb + c * 32, v);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (finish) gemm_epilogue<EPI, BN>(tb, row, row < M, n0, BN, ep);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

@@ -232,6 +232,10 @@ __global__ void positions_varlen_kernel(int s_txt, int grid_h, int grid_w, const
   pos[3 * t + 2] = a2;
 }
 
+__global__ void zero_ints_kernel(int* __restrict__ p, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0;
+}
+
 // Up to kLenChunk per-element text lengths carried by value into device memory
 // (no host-to-device copy, so the forward stays capturable in a CUDA graph).
 constexpr int kLenChunk = 64;

@@ -156,27 +156,34 @@ enum KernelBit : unsigned {
 
 constexpr int kStages = 4;
 
+// sk.partials == nullptr: no split tail (a caller without workspace).
 template <int BN, int EPI>
 int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint16_t* B, int M, int N, int K,
-             const EpiParams& ep, cudaStream_t st) {
+             const EpiParams& ep, cudaStream_t st, SplitScratch sk = SplitScratch{nullptr, nullptr}) {
   using L = GemmSmem<BN, kStages>;
+  static_assert(BN <= 256, "split partial slots hold 128 x 256 fp32");
   if (M <= 0) return ZI_OK;
   if (K % 64 != 0 || N % BN != 0 || K <= 0 || N <= 0) return ZI_ERR_SHAPE;
-  CUtensorMap ta, tb, tb64;
+  CUtensorMap ta, tb;
   ZI_TRY(make_map(&ta, A, uint64_t(K), uint64_t(M), uint64_t(K) * 2, 64, 128));
   ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, BN));
-  ZI_TRY(make_map(&tb64, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, 64));
   auto kern = gemm_bf16_tn_kernel<BN, kStages, EPI>;
   ZI_TRY(ensure_smem(dev, bit, kern, int(L::kBytes)));
   const int tiles = ((M + 127) / 128) * (N / BN);
-  const int grid = tiles < dev->sms ? tiles : dev->sms;
-  // sub-tiles must stay 64-column multiples; a QKV sub-tile must hold whole
-  // 128-wide heads; SwiGLU pairs 128 gate with 128 up columns, so no split
-  const int max_f = (EPI == EPI_SWIGLU || EPI == EPI_UNPATCH) ? 1 : (EPI == EPI_QKV ? 2 : BN / 64);
-  const TailSched sched = make_tail_sched(tiles, grid, max_f < 4 ? max_f : 4);
+  const TailSched sched = make_tail_sched(tiles, dev->sms, K / 64, sk.partials != nullptr);
+  int grid = tiles < dev->sms ? tiles : dev->sms;
+  if (sched.tail_items > grid) grid = sched.tail_items;  // fewer tiles than SMs, each cut along K
   prof_pre(st);
-  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, tb64, M, N, K, ep, sched);
+  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, N, K, ep, sched, sk);
   return launched(kind, st);
+}
+
+// Zeroes the split-tail counters of a workspace (once per forward; every tile's
+// finisher puts its counter back to zero).
+int clear_split(const SplitScratch& sk, cudaStream_t st) {
+  prof_pre(st);
+  zero_ints_kernel<<<1, 256, 0, st>>>(sk.counters, kSplitSlots);
+  return launched(ZI_KERNEL_SPLIT_CLEAR, st);
 }
 
 EpiParams epi_plain(void* out, int ldo) {
@@ -240,7 +247,7 @@ constexpr size_t kAlign = 1024;
 inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-  size_t mod, c, silu, hid, lens, pos, rope, x, h, qkv, att, o, u, tok, capn, total;
+  size_t mod, c, silu, hid, lens, pos, rope, x, h, qkv, att, o, u, tok, capn, split_cnt, split_part, total;
 };
 
 Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int mod_cols) {
@@ -268,6 +275,8 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.u = o; o = up(o + rows * Fp * 2);
   w.tok = o; o = up(o + (model ? size_t(batch) * s_img * size_t(4 * cfg.in_ch) * 2 : 0));
   w.capn = o; o = up(o + (model ? size_t(batch) * s_txt * size_t(cfg.cap_dim) * 2 : 0));
+  w.split_cnt = o; o = up(o + size_t(kSplitSlots) * 4);
+  w.split_part = o; o = up(o + size_t(kSplitSlots) * 128 * 256 * 4);
   w.total = o;
   return w;
 }
@@ -332,6 +341,7 @@ struct BlockCtx {
   int nseg;
   int seg_row0[2], seg_len[2];  // local rows
   const int* kv_len;  // [batch] keys of the last segment (valid text tokens), or null = all
+  SplitScratch split;  // split-tail scratch of the workspace (counters cleared)
 };
 
 int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
@@ -347,10 +357,12 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   eq.dim = D;
   eq.row_off = b.row_off;
   eq.map = b.map;
-  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st)));
+  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st,
+                                 b.split)));
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len,
                        b.kv_len, st));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D, epi_plain(b.o, D), st)));
+  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D,
+                                  epi_plain(b.o, D), st, b.split)));
   PostParams pa;
   memset(&pa, 0, sizeof(pa));
   pa.x_in = b.x_in;
@@ -371,9 +383,10 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   pa.eps = eps;
   pa.eps_ln = b.cfg->final_eps;
   ZI_TRY(run_post(pa, b.rows, st));
-  ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp, D, epi_plain(b.u, Fp),
-                                    st)));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp, epi_plain(b.o, D), st)));
+  ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp, D,
+                                    epi_plain(b.u, Fp), st, b.split)));
+  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp,
+                                  epi_plain(b.o, D), st, b.split)));
   PostParams pf = pa;
   pf.x_in = b.x_out;
   pf.g_post = b.w->g_ffn2;
@@ -653,6 +666,8 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.seg_row0[1] = 0;
   b.seg_len[1] = 1;
   b.kv_len = nullptr;
+  b.split = SplitScratch{reinterpret_cast<float4*>(ws + L.split_part), reinterpret_cast<int*>(ws + L.split_cnt)};
+  ZI_TRY(clear_split(b.split, st));
   ZI_TRY(run_rms_mod<float>(d_x_in, rows, D, w->g_attn1, b.mod, b.mod_ld, b.map, 0, cfg->norm_eps, b.h, st));
   const NextNormSpec none{NEXT_NONE, nullptr, nullptr, 0};
   return run_block(b, none, st);
@@ -733,6 +748,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   uint16_t* capn = reinterpret_cast<uint16_t*>(ws + L.capn);
   int* lens = h_txt_len ? reinterpret_cast<int*>(ws + L.lens) : nullptr;
   const RowMap map{rows_img, s_img, s_txt, h_txt_len ? S : 0};
+  const SplitScratch split{reinterpret_cast<float4*>(ws + L.split_part), reinterpret_cast<int*>(ws + L.split_cnt)};
   const float eps = cfg->norm_eps;
   int traced = 0;
   auto trace = [&]() -> int {
@@ -743,6 +759,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     return ZI_OK;
   };
 
+  ZI_TRY(clear_split(split, st));
   // timestep conditioning and every adaLN projection
   {
     float* hid = reinterpret_cast<float*>(ws + L.hid);
@@ -818,7 +835,8 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
                                  st));
     EpiParams ec = epi_plain(x + size_t(rows_img) * D, D);
     ec.bias = w->cap_b;
-    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, capn, w->cap_w, rows_txt, D, cfg->cap_dim, ec, st)));
+    ZI_TRY((run_gemm<256, EPI_F32_BIAS>(dev, BIT_GEMM_F32, ZI_KERNEL_GEMM_EMBED, capn, w->cap_w, rows_txt, D,
+                                        cfg->cap_dim, ec, st, split)));
     if (h_txt_len) {
       prof_pre(st);
       text_pad_kernel<<<dim3(s_txt, batch), 256, 0, st>>>(x + size_t(rows_img) * D, s_txt, D, lens, w->cap_pad);
@@ -834,6 +852,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   base.rope = rope;
   base.mod_ld = mod_ld;
   base.kv_len = lens;
+  base.split = split;
 
   auto segment_ctx = [&](int row_off, int nrows, int seglen) {
     BlockCtx b = base;
@@ -921,7 +940,8 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     ef.lat_c = cfg->in_ch;
     ef.lat_h = lat_h;
     ef.lat_w = lat_w;
-    ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, ZI_KERNEL_GEMM_FINAL, h, w->final_w, rows_img, 4 * cfg->in_ch, D, ef, st)));
+    ZI_TRY((run_gemm<64, EPI_UNPATCH>(dev, BIT_GEMM_UNPATCH, ZI_KERNEL_GEMM_FINAL, h, w->final_w, rows_img,
+                                      4 * cfg->in_ch, D, ef, st, split)));
   }
   return ZI_OK;
 }

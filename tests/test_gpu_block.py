@@ -64,6 +64,33 @@ def test_full_width_block_1152_tokens():
     run_block(dataclasses.replace(zi.FULL, n_noise=0, n_ctx=0, n_main=1), "layers.0", True, 1, 128, 32, 32, seed=3)
 
 
+def test_full_width_block_split_tails_deterministic():
+    """456 tokens (16 x 16 image + 200 text; 4 row tiles, the last ragged): every GEMM of
+    the block ends in a ragged wave cut along K (QKV and FFN-up in 4 pieces, out-proj
+    and FFN-down in 2), finished by whichever piece arrives last.  Parity with the
+    oracle, and two runs bit-identical (partials are added in a fixed order)."""
+    from stream_diffusion_transformer_b200 import model
+    d = dataclasses.replace(zi.FULL, n_noise=0, n_ctx=0, n_main=1)
+    cfg = model.make_config(d)
+    keys = model.block_keys("layers.0", True)
+    bits = zi.make_weights(d, seed=8, keys=keys, threads=8)
+    s_txt, gh, gw = 200, 16, 16
+    S = gh * gw + s_txt
+    x = zi.make_stream(d, 1, S, seed=8)
+    c = zi.make_cond(d, 1, seed=8)
+    blk = model.DeviceBlock(cfg, "layers.0", bits, True, "cuda")
+    pos = model.positions(s_txt, gh, gw)
+    xt, ct = torch.from_numpy(x).cuda(), torch.from_numpy(c).cuda()
+    out1 = model.block_forward(cfg, blk, ct, pos, xt).cpu().numpy()
+    out2 = model.block_forward(cfg, blk, ct, pos, xt).cpu().numpy()
+    np.testing.assert_array_equal(out1, out2)
+    W = ref.Weights(bits)
+    ang = ref.rope_angles(ref.position_ids(s_txt, gh, gw), d.rope_axes)
+    want = ref.block_forward(x[0].astype(np.float64), W, "layers.0", d, ang, c[0].astype(np.float64))
+    assert_parity(out1[0], want, rel=2e-2, cos=0.999, what="split-tail block")
+    assert_parity(out1[0] - x[0], want - x[0], rel=1.0, cos=0.99, what="split-tail block delta")
+
+
 def test_full_width_unmodulated_text_block():
     """A context-refiner-shaped block on 32 text tokens only (a single partial tile)."""
     d = dataclasses.replace(zi.FULL, n_noise=0, n_ctx=1, n_main=1)
