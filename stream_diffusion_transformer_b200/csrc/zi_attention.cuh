@@ -24,6 +24,13 @@
 // segment's end are masked to -inf.  An optional per-element key count for the
 // last segment (kv_len) drops that segment's trailing rows (padding) from the
 // keys: tiles wholly past it are never loaded, the tile it ends in is masked.
+//
+// Work units are (query-tile pair, head, batch element), one CTA each.  When the
+// units leave a ragged last wave of R < G (SM count) units and scratch is given,
+// those R units are cut along the keys into s pieces (s R <= G), one CTA per
+// piece: each piece writes its unnormalised O rows with their running max and
+// sum, and the piece that completes the unit's counter merges the pieces in
+// piece order (the same order whichever piece finishes) and writes the output.
 #pragma once
 #include "zi_common.cuh"
 
@@ -39,6 +46,11 @@ struct AttnParams {
   int q_tiles;      // query tiles per batch element (both segments)
   float scale_log2; // log2(e) / sqrt(head_dim)
   const int* kv_len;  // [batch] keys of the last segment per element, or null (= its seg_len)
+  int pairs, heads;   // units are (pair of query tiles, head, batch element), pair fastest
+  int full_units;     // units [0, full_units) run whole, one CTA each
+  int split_s;        // key pieces per remaining unit (1 = none)
+  float4* part;       // split scratch: kAttnSlotF4 float4 per piece (null = no split)
+  int* counters;      // one per split unit, zero on entry (the finisher resets it)
 };
 
 namespace attn {
@@ -51,6 +63,11 @@ constexpr uint32_t kQ0 = 0, kK0 = 2 * kTile, kV0 = 4 * kTile;
 constexpr uint32_t kBar = 6 * kTile;
 constexpr uint32_t kSmemBytes = kBar + 256 + 1024;
 constexpr uint32_t kColS = 0, kColO = 256;  // S_t at kColS + 128 t, O_t at kColO + 128 t
+constexpr int kMaxSplit = 4;
+// one piece's partial: O of both tiles [t][32 column quads][128 rows] float4, then
+// (m, l) of both tiles [t][128 rows] float2
+constexpr int kSlotOF4 = 2 * 32 * 128;
+constexpr int kSlotF4 = kSlotOF4 + 128;
 }  // namespace attn
 
 // Keys of the last segment of element b: kv_len[b] clamped to [1, seg_len], or all.
@@ -156,16 +173,28 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   uint64_t* p_full = bars + 11;  // [2 tiles]
   uint64_t* pv_done = bars + 13; // [2 tiles]
   uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* fin_bar = bars + 16;  // the softmax threads' meeting point (split pieces)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* fin_flag = abort_flag + 1;
 
   if (device_error_set()) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.y, b = blockIdx.z;
+  // which unit, and which piece of its keys, this CTA runs
+  int unit = blockIdx.x, piece = -1;
+  if (unit >= p.full_units) {
+    const int v = unit - p.full_units;
+    unit = p.full_units + v / p.split_s;
+    piece = v % p.split_s;
+  }
+  const int pair = unit % p.pairs, head = (unit / p.pairs) % p.heads, b = unit / (p.pairs * p.heads);
   const int last_keys = attn_last_keys(p, b);
   const int n_kv = p.nseg > 1 ? (p.seg_len[0] + 127) / 128 + (last_keys + 127) / 128 : (last_keys + 127) / 128;
-  const int tile_a = 2 * blockIdx.x;
-  const bool has_b = tile_a + 1 < p.q_tiles;  // CTA-uniform: the last CTA may hold one tile
+  // key tiles [j0, j0 + nj) of this CTA (all of them for a whole unit)
+  const int j0 = piece < 0 ? 0 : piece * n_kv / p.split_s;
+  const int nj = piece < 0 ? n_kv : (piece + 1) * n_kv / p.split_s - j0;
+  const int tile_a = 2 * pair;
+  const bool has_b = tile_a + 1 < p.q_tiles;  // CTA-uniform: the last pair may hold one tile
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -179,6 +208,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(fin_bar, has_b ? 256 : 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -220,11 +250,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const int col = kq ? colk : colv;
       uint32_t issued = 0;
       bool ok = true;
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = 0; j < nj; ++j) {
         const int bi = j & 1;
         const uint32_t r = uint32_t(j) >> 1;
         int kv0, kvn;
-        attn_tile_rows(p, b, j, last_keys, kv0, kvn);
+        attn_tile_rows(p, b, j0 + j, last_keys, kv0, kvn);
         if (!mbar_wait(&emptyb[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) { ok = false; break; }
         mbar_arrive_expect_tx(&fullb[bi], kTile);
         tma_load_2d(smem + base + bi * kTile, &tm, &fullb[bi], col, kv0);
@@ -287,8 +317,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       } else {
         ok = false;
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const bool more = j + 1 < n_kv;
+      for (int j = 0; j < nj && ok; ++j) {
+        const bool more = j + 1 < nj;
         if (more) {
           if (!wait_k(j + 1)) { ok = false; break; }
           tc_fence_after();
@@ -325,9 +355,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       float m_run = -INFINITY, l = 0.f;
       uint32_t s[128];
       bool ok = true;
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = 0; j < nj; ++j) {
         int kv0, kvn;
-        attn_tile_rows(p, b, j, last_keys, kv0, kvn);
+        attn_tile_rows(p, b, j0 + j, last_keys, kv0, kvn);
         if (!mbar_wait(&s_full[t], uint32_t(j) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -416,14 +446,113 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&p_full[t]);
       }
-      if (ok && mbar_wait(&pv_done[t], uint32_t(n_kv - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX)) {
-        tc_fence_after();
-        const float inv = 1.0f / l;
+      ok = ok && mbar_wait(&pv_done[t], uint32_t(nj - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX);
+      if (ok) tc_fence_after();
+      bool write = ok;
+      // merged output of a split unit: O = sum_k 2^(m_k - M) O_k, l = sum_k 2^(m_k - M) l_k
+      float mk[kMaxSplit], wk[kMaxSplit];
+      float inv = 1.0f;
+      const float4* slot0 = nullptr;
+      if (ok && piece >= 0) {
+        const int first = (unit - p.full_units) * p.split_s;  // slot of piece 0
+        slot0 = p.part + size_t(first) * kSlotF4;
+        float4* mine = p.part + size_t(first + piece) * kSlotF4;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32_sync(o_addr + c * 32, o);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            __stcg(mine + (t * 32 + c * 8 + k) * 128 + i,
+                   make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                               __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3])));
+        }
+        __stcg(reinterpret_cast<float2*>(mine + kSlotOF4) + t * 128 + i, make_float2(m_run, l));
+        __threadfence();
+        mbar_arrive(fin_bar);
+        ok = mbar_wait(fin_bar, 0, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX);
+        if (ok && threadIdx.x == 0) {
+          const int u = unit - p.full_units;
+          const bool last = atomicAdd(&p.counters[u], 1) == p.split_s - 1;
+          if (last) p.counters[u] = 0;  // ready for the next launch
+          *fin_flag = last ? 1 : 0;
+        }
+        if (ok) {
+          mbar_arrive(fin_bar);
+          ok = mbar_wait(fin_bar, 1, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX);
+        }
+        write = ok && *fin_flag != 0;
+        if (write) {
+          __threadfence();
+          float M = -INFINITY, L = 0.f;
+#pragma unroll
+          for (int k = 0; k < kMaxSplit; ++k) {
+            mk[k] = -INFINITY;
+            float lk = 0.f;
+            if (k < p.split_s) {
+              if (k == piece) {
+                mk[k] = m_run;
+                lk = l;
+              } else {
+                const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot0 + size_t(k) * kSlotF4 + kSlotOF4) +
+                                         t * 128 + i);
+                mk[k] = ml.x;
+                lk = ml.y;
+              }
+            }
+            M = fmaxf(M, mk[k]);
+            wk[k] = lk;  // l_k for now
+          }
+#pragma unroll
+          for (int k = 0; k < kMaxSplit; ++k) {
+            const float lk = wk[k];
+            wk[k] = k < p.split_s ? fast_exp2(mk[k] - M) : 0.f;
+            if (k < p.split_s) L = k == 0 ? wk[k] * lk : fmaf(wk[k], lk, L);
+          }
+          inv = 1.0f / L;
+        }
+      } else if (ok) {
+        inv = 1.0f / l;
+      }
+      if (write) {
         uint16_t* orow = p.out + size_t(q_row0 + i) * p.ldo + head * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32_sync(o_addr + c * 32, o);
+          if (piece >= 0) {
+            // the other pieces' 32 columns, loaded together before any is used
+            float4 pp[kMaxSplit][8];
+#pragma unroll
+            for (int k = 0; k < kMaxSplit; ++k) {
+              const bool need = k < p.split_s && k != piece;
+              const float4* src = slot0 + size_t(k) * kSlotF4 + (t * 32 + c * 8) * 128 + i;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) pp[k][e] = need ? __ldcg(src + e * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int k = 0; k < kMaxSplit; ++k) {
+                if (k < p.split_s) {
+                  const float4 ok4 = k == piece ? make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                              __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]))
+                                                : pp[k][e];
+                  if (k == 0) {
+                    acc = make_float4(wk[0] * ok4.x, wk[0] * ok4.y, wk[0] * ok4.z, wk[0] * ok4.w);
+                  } else {
+                    acc = make_float4(fmaf(wk[k], ok4.x, acc.x), fmaf(wk[k], ok4.y, acc.y), fmaf(wk[k], ok4.z, acc.z),
+                                      fmaf(wk[k], ok4.w, acc.w));
+                  }
+                }
+              }
+              o[4 * e] = __float_as_uint(acc.x);
+              o[4 * e + 1] = __float_as_uint(acc.y);
+              o[4 * e + 2] = __float_as_uint(acc.z);
+              o[4 * e + 3] = __float_as_uint(acc.w);
+            }
+          }
           if (i < q_valid) {
             uint4* d = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll

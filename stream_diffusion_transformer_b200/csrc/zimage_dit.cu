@@ -178,6 +178,8 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint
   return launched(kind, st);
 }
 
+static_assert(size_t(attn::kSlotF4) * 16 >= size_t(128) * 256 * 4, "a split slot holds a GEMM tile partial");
+
 // Zeroes the split-tail counters of a workspace (once per forward; every tile's
 // finisher puts its counter back to zero).
 int clear_split(const SplitScratch& sk, cudaStream_t st) {
@@ -197,8 +199,10 @@ EpiParams epi_plain(void* out, int ldo) {
 
 // ---------------------------------------------------------------- attention
 
+// sk.partials == nullptr: no split of the ragged last wave.
 int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out, int dim, int heads, int batch,
-                  int nseg, const int* row0, const int* len, const int* kv_len, cudaStream_t st) {
+                  int nseg, const int* row0, const int* len, const int* kv_len, cudaStream_t st,
+                  SplitScratch sk = SplitScratch{nullptr, nullptr}) {
   CUtensorMap tm;
   ZI_TRY(make_map(&tm, qkv, uint64_t(3 * dim), uint64_t(qkv_rows), uint64_t(3 * dim) * 2, 64, 128));
   ZI_TRY(ensure_smem(dev, BIT_ATTN, attention_kernel, int(attn::kSmemBytes)));
@@ -217,7 +221,28 @@ int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(128.0));
   p.q_tiles = qt;
   p.kv_len = kv_len;
-  dim3 grid((qt + 1) / 2, heads, batch);  // two query tiles per CTA
+  p.pairs = (qt + 1) / 2;  // two query tiles per unit
+  p.heads = heads;
+  const long long units = static_cast<long long>(p.pairs) * heads * batch;
+  if (units > 0x7fffffffLL / attn::kMaxSplit) return ZI_ERR_SHAPE;
+  p.full_units = int(units);
+  p.split_s = 1;
+  const int G = dev->sms;
+  const int rest = int(units % G);
+  // fewest key tiles any element can have (each piece needs one)
+  const int min_kv = (nseg > 1 ? (len[0] + 127) / 128 : 0) + (kv_len ? 1 : (len[nseg - 1] + 127) / 128);
+  if (sk.partials && rest > 0 && G <= kSplitSlots) {
+    int f = G / rest;
+    if (f > attn::kMaxSplit) f = attn::kMaxSplit;
+    if (f > min_kv) f = min_kv;
+    if (f >= 2) {
+      p.full_units = int(units) - rest;
+      p.split_s = f;
+      p.part = sk.partials;
+      p.counters = sk.counters;
+    }
+  }
+  const int grid = p.full_units + (int(units) - p.full_units) * p.split_s;
   prof_pre(st);
   attention_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(tm, p);
   return launched(ZI_KERNEL_ATTENTION, st);
@@ -276,7 +301,9 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.tok = o; o = up(o + (model ? size_t(batch) * s_img * size_t(4 * cfg.in_ch) * 2 : 0));
   w.capn = o; o = up(o + (model ? size_t(batch) * s_txt * size_t(cfg.cap_dim) * 2 : 0));
   w.split_cnt = o; o = up(o + size_t(kSplitSlots) * 4);
-  w.split_part = o; o = up(o + size_t(kSplitSlots) * 128 * 256 * 4);
+  // partial slots of the split tails: a GEMM tile (128 x 256 fp32) or an attention
+  // piece (O of two query tiles plus their row max and sum), whichever is larger
+  w.split_part = o; o = up(o + size_t(kSplitSlots) * size_t(attn::kSlotF4) * 16);
   w.total = o;
   return w;
 }
@@ -360,7 +387,7 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st,
                                  b.split)));
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len,
-                       b.kv_len, st));
+                       b.kv_len, st, b.split));
   ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D,
                                   epi_plain(b.o, D), st, b.split)));
   PostParams pa;
