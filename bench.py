@@ -357,11 +357,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      ("gemm_ffn_down", 2.0 * S * d.dim * d.ffn)):
         m = statistics.mean(main_block_launches(kind))
         per_kernel_roof[kind] = {"ms_per_launch": m, "tflops": fl / (m * 1e-3) / 1e12,
-                                 "frac": fl / (m * 1e-3) / 1e12 / peak_tensor}
+                                 "frac": fl / (m * 1e-3) / 1e12 / peak_tensor, "traffic": recorded_traffic(kind)}
     for kind, bytes_per_row in (("post_norm_residual", 4 * d.dim * 2 + 2 * d.dim * 2),):
         m = statistics.mean(main_block_launches(kind))
         gbs = bytes_per_row * S / (m * 1e-3) / 1e9
-        per_kernel_roof[kind] = {"ms_per_launch": m, "gbs": gbs, "frac": gbs / float(peaks["hbm_gbs"])}
+        per_kernel_roof[kind] = {"ms_per_launch": m, "gbs": gbs, "frac": gbs / float(peaks["hbm_gbs"]),
+                                 "algorithmic_bytes_per_launch": bytes_per_row * S, "traffic": recorded_traffic(kind)}
 
     clk = clocks.summary()
     value = flops * world * args.steps / (ms * 1e-3) / 1e12
@@ -454,20 +455,22 @@ def run_loop_workload(args, n_steps: int = 8, s_txt: int = 128):
     dit = model.DiT(model.make_config(d), lambda keys: zi.make_weights(d, seed=SEED, keys=keys, threads=threads))
     lat = torch.from_numpy(zi.make_latent(d, 1, LAT_H, LAT_W, seed=SEED)).cuda()
     txt = torch.from_numpy(zi.make_text(d, 1, s_txt, seed=SEED).view(np.int16)).cuda().view(torch.bfloat16)
+    graph = model.DenoiseGraph(dit, tuple(lat.shape), txt, n_steps=n_steps)  # the loop as one CUDA graph
     for _ in range(args.warmup):
-        dit.denoise(lat, txt, n_steps=n_steps)
+        graph.run(lat)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(0) as clocks:
         e0.record()
         for _ in range(args.steps):
-            x = dit.denoise(lat, txt, n_steps=n_steps)
+            x = graph.run(lat)
         e1.record()
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     s_img = (LAT_H // 2) * (LAT_W // 2)
     fl = n_steps * forward_flops(d, s_img, s_txt)
-    print(json.dumps({"workload": f"8-step Turbo loop, 1024x1024, {s_img} + {s_txt} tokens, shift 3",
+    print(json.dumps({"workload": f"8-step Turbo loop, 1024x1024, {s_img} + {s_txt} tokens, shift 3, "
+                                  "replayed as one CUDA graph",
                       "ms_per_loop": ms, "ms_per_forward": ms / n_steps, "value": fl / (ms * 1e-3) / 1e12,
                       "unit": "TFLOP/s", "steps": args.steps, "warmup": args.warmup,
                       "finite": bool(torch.isfinite(x).all().item()), "device_status": abi.device_status(),

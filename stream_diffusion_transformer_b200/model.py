@@ -210,6 +210,37 @@ class DiT:
         return out
 
 
+class DenoiseGraph:
+    """DiT.denoise captured once as a CUDA graph and replayed: all n_steps forwards,
+    their Euler steps (sigmas baked in) and, with guidance, the CFG combines, for
+    one fixed latent shape and fixed text features (read in place by every replay:
+    change them with copy_() to condition on other text).  run(latent) copies the latent
+    into the graph's input buffer, replays, and returns the graph's output tensor
+    (overwritten by the next run)."""
+
+    def __init__(self, dit: "DiT", latent_shape, txt: torch.Tensor, n_steps: int = 8, shift: float = 3.0,
+                 guidance: Optional[float] = None, txt_uncond: Optional[torch.Tensor] = None,
+                 txt_len: Optional[Sequence[int]] = None, txt_uncond_len: Optional[Sequence[int]] = None):
+        self.x0 = torch.zeros(tuple(latent_shape), dtype=torch.float32, device=dit.device)
+        # the graph reads the text features by address: hold them for its lifetime
+        self.txt, self.txt_uncond = txt, txt_uncond
+        kw = dict(n_steps=n_steps, shift=shift, guidance=guidance, txt_uncond=txt_uncond, txt_len=txt_len,
+                  txt_uncond_len=txt_uncond_len)
+        # one eager run first: kernel attributes are set and the workspace exists
+        # before capture (neither may happen while the stream is being captured)
+        dit.denoise(self.x0, txt, **kw)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.out = dit.denoise(self.x0, txt, **kw)
+        torch.cuda.synchronize()
+
+    def run(self, latent: torch.Tensor) -> torch.Tensor:
+        self.x0.copy_(latent)
+        self.graph.replay()
+        return self.out
+
+
 def forward_trace(dit: "DiT", latent: torch.Tensor, t: torch.Tensor, txt: torch.Tensor):
     """DiT.forward that also returns the residual stream after every block:
     (out, trace fp32 [n_blocks, rows, dim]) with rows = image rows then text rows."""
