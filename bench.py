@@ -525,6 +525,59 @@ def run_cfg_workload(args):
                       "clocks": clocks.summary()}), flush=True)
 
 
+def run_fp8_workload(args):
+    """The metric's forward (4,128 tokens at 1024x1024, batch 1) with every block's QKV
+    and FFN w1|w3 projections in e4m3 (per-row scales, tcgen05 kind::f8f6f4); the other
+    steps stay as in the bf16 forward.  FLOPs are counted as for the bf16 forward."""
+    import torch
+
+    from stream_diffusion_transformer_b200 import abi, model
+
+    d = zi.FULL
+    threads = max(1, min(32, (os.cpu_count() or 8)))
+    dit = model.DiT(model.make_config(d), lambda keys: zi.make_weights(d, seed=SEED, keys=keys, threads=threads),
+                    fp8=True)
+    lat = torch.from_numpy(zi.make_latent(d, 1, LAT_H, LAT_W, seed=SEED)).cuda()
+    txt = torch.from_numpy(zi.make_text(d, 1, S_TXT, seed=SEED).view(np.int16)).cuda().view(torch.bfloat16)
+    tt = torch.full((1,), T_VALUE, dtype=torch.float32, device="cuda")
+    out = torch.empty_like(lat)
+    for _ in range(args.warmup):
+        dit.forward(lat, tt, txt, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks, abi.Profile(capacity=300 * args.steps + 16) as prof:
+        e0.record()
+        for _ in range(args.steps):
+            dit.forward(lat, tt, txt, out)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    s_img = (LAT_H // 2) * (LAT_W // 2)
+    S = s_img + S_TXT
+    fl = forward_flops(d, s_img, S_TXT)
+    peaks, peak_src = load_peaks()
+    peak_f8 = 2.0 * float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))  # e4m3 = 2x bf16 (nominal ratio)
+    per_step = len(prof.kinds) // args.steps
+    roof = {}
+    for kind, kfl in (("gemm_qkv_qknorm_rope", 6.0 * S * d.dim ** 2), ("gemm_ffn_up_swiglu", 4.0 * S * d.dim * d.ffn)):
+        ms_k = []
+        for sidx in range(args.steps):
+            seq = [m for k, m in zip(prof.kinds[sidx * per_step:(sidx + 1) * per_step],
+                                     prof.ms[sidx * per_step:(sidx + 1) * per_step]) if k == kind]
+            ms_k += seq[-d.n_main:]
+        m = statistics.mean(ms_k)
+        roof[kind] = {"ms_per_launch": m, "tflops": kfl / (m * 1e-3) / 1e12, "peak": peak_f8,
+                      "frac": kfl / (m * 1e-3) / 1e12 / peak_f8,
+                      "peak_source": f"{peak_src} bf16 sustained x 2 (nominal e4m3 / bf16 ratio)"}
+    by = {k: {"launches": v[0], "ms": round(v[1] / args.steps, 3)} for k, v in prof.by_kernel().items()}
+    print(json.dumps({"workload": f"e4m3 QKV + FFN-up projections, 1024x1024, {s_img} + {S_TXT} tokens, batch 1",
+                      "ms_per_step": ms, "value": fl / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "dtype": "e4m3 (QKV, FFN w1|w3) + bf16", "flops_per_step": fl, "steps": args.steps,
+                      "warmup": args.warmup, "kernel_rooflines": roof, "kernels_ms_per_step": by,
+                      "finite": bool(torch.isfinite(out).all().item()), "device_status": abi.device_status(),
+                      "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -532,7 +585,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg"], default="forward",
+    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
                          "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens; "
                          "cfg: one guidance step at 2048x2048, batch 2 x 16,896 tokens")
@@ -545,6 +598,9 @@ def main():
         return
     if args.workload == "cfg":
         run_cfg_workload(args)
+        return
+    if args.workload == "fp8":
+        run_fp8_workload(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

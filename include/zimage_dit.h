@@ -105,6 +105,16 @@ typedef struct zi_block_weights {
   const uint16_t* g_k;     /* [head_dim] */
   const uint16_t* w_ada;   /* [4D, min(D,256)] adaLN linear, or NULL for an unmodulated block */
   const uint16_t* b_ada;   /* [4D] its bias (NULL iff w_ada is NULL) */
+  /* Optional e4m3 projections (all four, or all NULL).  When set, the block's QKV
+   * and FFN w1|w3 projections run on the tensor cores in e4m3 (kind::f8f6f4)
+   * from these instead of w_qkv / w13, and the norms feeding them emit e4m3
+   * activations with one scale per token row (zi_quantize_rows_e4m3 gives the
+   * recipe; its header comment states it).  The pages' quantised builds (ostris
+   * "Z-Image", "Specifics"; H3ddle "What was changed, and why") are the prior art. */
+  const uint8_t* w_qkv8;   /* [3D, D] e4m3 codes of w_qkv, one scale per row ... */
+  const float* s_qkv;      /* [3D] ... these (zi_quantize_rows_e4m3 of w_qkv) */
+  const uint8_t* w13_8;    /* [2Fp, D] e4m3 codes of w13 */
+  const float* s_13;       /* [2Fp] */
 } zi_block_weights;
 
 /* Weights of the whole transformer.  The block arrays are HOST arrays (of
@@ -293,6 +303,23 @@ ZI_API int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, floa
 ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k,
                         zi_stream_t stream);
 
+/* Per-row e4m3 quantisation (OCP e4m3: bias 7, 3 mantissa bits, max 448):
+ *   s[r] = amax_r / 448 (fp32), q[r][k] = e4m3(x[r][k] * (448 / amax_r)), the
+ *   product formed in fp32, rounded to nearest even, saturating at +-448; a row of
+ *   zeros gets s = 1 and zero codes.  The same recipe the norms use for e4m3 blocks.
+ *   d_x   [rows, cols] fp32 (x_bf16 = 0) or bf16 (x_bf16 = 1), contiguous
+ *   d_q   [rows, cols] uint8 codes;  d_s [rows] fp32 scales
+ * cols % 4 == 0 and cols <= 4096 (ZI_ERR_SHAPE otherwise); 16-byte aligned pointers.
+ * Weights for e4m3 blocks are made with it (rows = output channels). */
+ZI_API int zi_quantize_rows_e4m3(const void* d_x, int x_bf16, int rows, int cols, uint8_t* d_q, float* d_s,
+                                 zi_stream_t stream);
+
+/* C[M, N] = bf16( sa[m] sb[n] sum_k A[m, k] B[n, k] ), A and B e4m3 codes (row-major,
+ * K contiguous), sa [M] / sb [N] their per-row scales; fp32 accumulation on
+ * tcgen05 (kind::f8f6f4).  K % 128 == 0, N % 256 == 0. */
+ZI_API int zi_gemm_e4m3(const uint8_t* d_a, const float* d_sa, const uint8_t* d_b, const float* d_sb, uint16_t* d_c,
+                        int m, int n, int k, zi_stream_t stream);
+
 /* Non-causal softmax(q k^T / sqrt(128)) v per head over seq tokens per batch element.
  * d_qkv bf16 [batch*seq, 3*heads*128] (q | k | v, head h at columns h*128 of each);
  * d_out bf16 [batch*seq, heads*128]. */
@@ -326,7 +353,8 @@ enum zi_kernel_kind {
   ZI_KERNEL_EULER = 15,         /* Euler / CFG step */
   ZI_KERNEL_GEMM = 16,          /* zi_gemm_bf16 */
   ZI_KERNEL_TEXT_PAD = 17,      /* cap_pad_token into padded text rows */
-  ZI_KERNEL_SPLIT_CLEAR = 18    /* zero the GEMM split-tail counters (once per forward) */
+  ZI_KERNEL_SPLIT_CLEAR = 18,   /* zero the GEMM split-tail counters (once per forward) */
+  ZI_KERNEL_QUANTIZE = 19       /* zi_quantize_rows_e4m3 */
 };
 
 /* Start recording launch timings on this host thread: from the next kernel the

@@ -34,7 +34,7 @@ class ZiConfig(ctypes.Structure):
 
 
 BLOCK_FIELDS = ("w_qkv", "w_out", "w13", "w2", "g_attn1", "g_attn2", "g_ffn1", "g_ffn2", "g_q", "g_k",
-                "w_ada", "b_ada")
+                "w_ada", "b_ada", "w_qkv8", "s_qkv", "w13_8", "s_13")
 
 
 class ZiBlockWeights(ctypes.Structure):
@@ -78,6 +78,8 @@ _SIGS = {
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
     "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_quantize_rows_e4m3": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "zi_gemm_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_attention_varlen": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_profile_begin": (c_int, [c_int]),
     "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),
@@ -162,7 +164,7 @@ KERNEL_NAMES = {
     1: "gemm_qkv_qknorm_rope", 2: "attention", 3: "gemm_out_proj", 4: "gemm_ffn_up_swiglu",
     5: "gemm_ffn_down", 6: "post_norm_residual", 7: "pre_norm", 8: "adaln_gemv", 9: "timestep_mlp",
     10: "rope_table", 11: "positions", 12: "patchify", 13: "gemm_embed", 14: "gemm_final_unpatchify",
-    15: "euler", 16: "gemm", 17: "text_pad", 18: "split_clear",
+    15: "euler", 16: "gemm", 17: "text_pad", 18: "split_clear", 19: "quantize_e4m3",
 }
 
 

@@ -52,6 +52,8 @@ struct EpiParams {
   int row_off;             // global row of local row 0 (for RowMap)
   RowMap map;
   int s_img, grid_w, lat_c, lat_h, lat_w;  // EPI_UNPATCH
+  const float* a_scale;  // e4m3 operands: per-row scale of A [M] ...
+  const float* b_scale;  // ... and of B [N] (per output column)
 };
 
 template <int BN, int STAGES>
@@ -81,16 +83,32 @@ ZI_DEV void store_bf16x32(uint16_t* dst, const float* v) {
 
 // Epilogue of one tile of `width` columns (width <= BN, a multiple of 64)
 // starting at output column n0.
-template <int EPI, int BN>
+// acc[i] *= sa * b_scale[col + i] for 32 accumulator columns (e4m3 operands).
+ZI_DEV void scale_acc32(uint32_t* v, float sa, const float* b_scale, int col) {
+  const float4* bs = reinterpret_cast<const float4*>(b_scale + col);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 w = __ldg(bs + q);
+    v[4 * q] = __float_as_uint(__uint_as_float(v[4 * q]) * (sa * w.x));
+    v[4 * q + 1] = __float_as_uint(__uint_as_float(v[4 * q + 1]) * (sa * w.y));
+    v[4 * q + 2] = __float_as_uint(__uint_as_float(v[4 * q + 2]) * (sa * w.z));
+    v[4 * q + 3] = __float_as_uint(__uint_as_float(v[4 * q + 3]) * (sa * w.w));
+  }
+}
+
+template <int EPI, int BN, bool F8>
 ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int width, const EpiParams& ep) {
+  static_assert(!F8 || EPI == EPI_BF16 || EPI == EPI_QKV || EPI == EPI_SWIGLU, "e4m3 epilogues: bf16, QKV, SwiGLU");
   uint32_t v[32];
   float f[32];
+  const float sa = (F8 && row_ok) ? __ldg(ep.a_scale + row) : 1.f;
   if constexpr (EPI == EPI_BF16 || EPI == EPI_F32_BIAS) {
 #pragma unroll 1
     for (int c = 0; c < width / 32; ++c) {
       tmem_ld32_sync(tbase + c * 32, v);
       if (row_ok) {
         const int col = n0 + c * 32;
+        if constexpr (F8) scale_acc32(v, sa, ep.b_scale, col);
         if constexpr (EPI == EPI_BF16) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
@@ -124,6 +142,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
       for (int c = 0; c < width / 32; ++c) {
         tmem_ld32_sync(tbase + c * 32, v);
         if (row_ok) {
+          if constexpr (F8) scale_acc32(v, sa, ep.b_scale, n0 + c * 32);
 #pragma unroll
           for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
           store_bf16x32(orow + n0 + c * 32, f);
@@ -140,6 +159,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         tmem_ld32_sync(tbase + hh * 128 + c * 32, v);
+        if constexpr (F8) scale_acc32(v, sa, ep.b_scale, n0 + hh * 128 + c * 32);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float x = __uint_as_float(v[i]);
@@ -151,6 +171,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
       for (int c = 0; c < 4; ++c) {
         tmem_ld32_sync(tbase + hh * 128 + c * 32, v);
         if (row_ok) {
+          if constexpr (F8) scale_acc32(v, sa, ep.b_scale, n0 + hh * 128 + c * 32);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int d0 = c * 32 + 2 * i;
@@ -176,6 +197,10 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
       reg_fence32(v);
       reg_fence32(u);
       if (row_ok) {
+        if constexpr (F8) {
+          scale_acc32(v, sa, ep.b_scale, n0 + c * 32);
+          scale_acc32(u, sa, ep.b_scale, n0 + 128 + c * 32);
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float gt = __uint_as_float(v[i]);
@@ -284,12 +309,15 @@ struct SplitScratch {
   int* counters;
 };
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
-    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                        int N, int K, EpiParams ep, TailSched sched, SplitScratch sk) {
+// The persistent GEMM, for bf16 operands (F8 = false: kind::f16, 64 elements per
+// 128-byte smem row) or e4m3 operands (F8 = true: kind::f8f6f4, 128 elements per
+// row, accumulator scaled by ep.a_scale[row] * ep.b_scale[col] in the epilogue).
+// The stage layout, swizzle and MMA count per stage (4) are the same for both.
+template <int BN, int STAGES, int EPI, bool F8>
+ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, const EpiParams& ep,
+                         const TailSched& sched, const SplitScratch& sk) {
   using L = GemmSmem<BN, STAGES>;
-  constexpr int BM = 128, BK = 64;
+  constexpr int BM = 128, BK = F8 ? 128 : 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -372,7 +400,7 @@ __global__ void __launch_bounds__(192, 1)
       int local = 0;
       bool ok = true;
       WorkWalker walk(sched, blockIdx.x);
-      const uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, false, false);
       while (ok && walk.next(wi)) {
         const int acc = local & 1;
         const uint32_t u = uint32_t(local) >> 1;
@@ -393,9 +421,14 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t a_addr = smem_u32(smem + s * L::kStage);
           const uint32_t b_addr = a_addr + L::kABytes;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            tc_mma(d, smem_desc_sw128(a_addr + k * 32, 16), smem_desc_sw128(b_addr + k * 32, 16), idesc,
-                   (kb != wi.kb0 || k != 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per MMA: 16 bf16 or 32 e4m3 elements
+            const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16), bd = smem_desc_sw128(b_addr + k * 32, 16);
+            const uint32_t acc_in = (kb != wi.kb0 || k != 0) ? 1u : 0u;
+            if constexpr (F8) {
+              tc_mma_f8(d, ad, bd, idesc, acc_in);
+            } else {
+              tc_mma(d, ad, bd, idesc, acc_in);
+            }
           }
           tc_commit(&empty[s]);
           ++it;
@@ -496,7 +529,7 @@ __global__ void __launch_bounds__(192, 1)
           tmem_wait_st();
         }
       }
-      if (finish) gemm_epilogue<EPI, BN>(tb, row, row < M, n0, BN, ep);
+      if (finish) gemm_epilogue<EPI, BN, F8>(tb, row, row < M, n0, BN, ep);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -507,6 +540,20 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
   }
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                        EpiParams ep, TailSched sched, SplitScratch sk) {
+  gemm_tn_body<BN, STAGES, EPI, false>(tmA, tmB, M, ep, sched, sk);
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_e4m3_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                        EpiParams ep, TailSched sched, SplitScratch sk) {
+  gemm_tn_body<BN, STAGES, EPI, true>(tmA, tmB, M, ep, sched, sk);
 }
 
 }  // namespace zi

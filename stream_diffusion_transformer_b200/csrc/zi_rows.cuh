@@ -23,6 +23,44 @@ ZI_DEV float block_sum(float v, float* red) {
   return t;
 }
 
+ZI_DEV float block_max(float v, float* red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = red[0];
+#pragma unroll
+  for (int i = 1; i < kRowThreads / 32; ++i) t = fmaxf(t, red[i]);
+  return t;
+}
+
+// Stores a row held by the CTA (y[k] for vector i = threadIdx.x + k * kRowThreads <
+// nvec) as e4m3 codes with one fp32 scale: amax / 448, codes of y * (448 / amax)
+// (round to nearest even, saturating); an all-zero row gets scale 1 and zero codes.
+// Every thread of the CTA must call it.
+ZI_DEV void store_row_e4m3(const float4* y, int nvec, float* red, uint8_t* q, float* scale) {
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < nvec) m = fmaxf(m, fmaxf(fmaxf(fabsf(y[k].x), fabsf(y[k].y)), fmaxf(fabsf(y[k].z), fabsf(y[k].w))));
+  }
+  const float amax = block_max(m, red);
+  const bool zero = amax == 0.f;
+  const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
+  if (threadIdx.x == 0) *scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    if (i < nvec) {
+      const float4 v = y[k];
+      reinterpret_cast<uint32_t*>(q)[i] =
+          zero ? 0u : pack_e4m3x4(__fmul_rn(v.x, inv), __fmul_rn(v.y, inv), __fmul_rn(v.z, inv), __fmul_rn(v.w, inv));
+    }
+  }
+}
+
 ZI_DEV float4 ld_bf16x4(const uint16_t* p) {
   const uint2 u = *reinterpret_cast<const uint2*>(p);
   return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
@@ -38,13 +76,15 @@ ZI_DEV void st_bf16x4(uint16_t* p, float4 v) {
 
 // h[row] = bf16( gain * x / sqrt(mean(x^2) + eps) * mscale[batch(row)] )
 // x is fp32 (TIn = float) or bf16 (TIn = uint16_t); mscale holds 1 + scale as the
-// adaLN kernel stores it, or is null (no modulation).
+// adaLN kernel stores it, or is null (no modulation).  With hq non-null the row
+// is written as e4m3 codes into hq [rows][D] with its scale in hs[row] instead.
 template <typename TIn>
 __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restrict__ x, int D,
                                                               const uint16_t* __restrict__ gain,
                                                               const float* __restrict__ scale, int scale_ld,
                                                               RowMap map, int row_off, float eps,
-                                                              uint16_t* __restrict__ h) {
+                                                              uint16_t* __restrict__ h, uint8_t* __restrict__ hq,
+                                                              float* __restrict__ hs) {
   __shared__ float red[kRowThreads / 32];
   const int row = blockIdx.x;
   const int nvec = D >> 2;
@@ -72,11 +112,37 @@ __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restr
       const float4 g = ld_bf16x4(gain + 4 * i);
       float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
       if (sc) m = reinterpret_cast<const float4*>(sc)[i];
-      st_bf16x4(h + size_t(row) * D + 4 * i,
-                make_float4(v[k].x * r * g.x * m.x, v[k].y * r * g.y * m.y, v[k].z * r * g.z * m.z,
-                            v[k].w * r * g.w * m.w));
+      v[k] = make_float4(v[k].x * r * g.x * m.x, v[k].y * r * g.y * m.y, v[k].z * r * g.z * m.z,
+                         v[k].w * r * g.w * m.w);
+      if (!hq) st_bf16x4(h + size_t(row) * D + 4 * i, v[k]);
     }
   }
+  if (hq) store_row_e4m3(v, nvec, red, hq + size_t(row) * D, hs + row);
+}
+
+// Per-row e4m3 quantisation of x [rows][D] (fp32 or bf16): q [rows][D] codes and
+// s [rows] scales, as store_row_e4m3 forms them.  One CTA per row.
+template <typename TIn>
+__global__ void __launch_bounds__(kRowThreads) quantize_rows_e4m3_kernel(const TIn* __restrict__ x, int D,
+                                                                         uint8_t* __restrict__ q,
+                                                                         float* __restrict__ s) {
+  __shared__ float red[kRowThreads / 32];
+  const int row = blockIdx.x;
+  const int nvec = D >> 2;
+  float4 v[kRowMaxVec];
+#pragma unroll
+  for (int k = 0; k < kRowMaxVec; ++k) {
+    const int i = threadIdx.x + k * kRowThreads;
+    v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < nvec) {
+      if constexpr (sizeof(TIn) == 4) {
+        v[k] = reinterpret_cast<const float4*>(x + size_t(row) * D)[i];
+      } else {
+        v[k] = ld_bf16x4(reinterpret_cast<const uint16_t*>(x) + size_t(row) * D + 4 * i);
+      }
+    }
+  }
+  store_row_e4m3(v, nvec, red, q + size_t(row) * D, s + row);
 }
 
 enum NextNorm : int { NEXT_NONE = 0, NEXT_RMS = 1, NEXT_LAYERNORM = 2 };
@@ -101,6 +167,8 @@ struct PostParams {
   int scale_ld;
   int next_rows;
   uint16_t* h;
+  uint8_t* hq;  // non-null: the next norm's output as e4m3 codes [rows][D] ...
+  float* hs;    // ... with one scale per row (NEXT_RMS only)
   RowMap map;
   int row_off;  // global row of local row 0 (for the batch lookup)
   int D;
@@ -177,11 +245,12 @@ __global__ void __launch_bounds__(kRowThreads) post_residual_kernel(PostParams p
       if (p.next == NEXT_RMS) g = ld_bf16x4(p.g_next + 4 * i);
       float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
       if (sc) m = reinterpret_cast<const float4*>(sc)[i];
-      st_bf16x4(p.h + size_t(row) * D + 4 * i,
-                make_float4((v[k].x - mu) * r * g.x * m.x, (v[k].y - mu) * r * g.y * m.y,
-                            (v[k].z - mu) * r * g.z * m.z, (v[k].w - mu) * r * g.w * m.w));
+      v[k] = make_float4((v[k].x - mu) * r * g.x * m.x, (v[k].y - mu) * r * g.y * m.y,
+                         (v[k].z - mu) * r * g.z * m.z, (v[k].w - mu) * r * g.w * m.w);
+      if (!p.hq) st_bf16x4(p.h + size_t(row) * D + 4 * i, v[k]);
     }
   }
+  if (p.hq) store_row_e4m3(v, nvec, red, p.hq + size_t(row) * D, p.hs + row);
 }
 
 // Position ids of one sequence [image tokens; text tokens]:

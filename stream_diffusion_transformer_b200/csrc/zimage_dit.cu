@@ -87,7 +87,8 @@ int encode_fn(EncodeTiledFn* out) {
 // 2-D bf16 map over a row-major [outer, inner] matrix with rows `row_bytes`
 // apart; box = box_inner x box_outer elements, 128-byte swizzle, zero fill.
 int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-             uint32_t box_inner, uint32_t box_outer) {
+             uint32_t box_inner, uint32_t box_outer,
+             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc;
   if (encode_fn(&enc) != ZI_OK) return ZI_ERR_CUDA;
   if ((reinterpret_cast<uintptr_t>(base) & 15u) || (row_bytes & 15u)) return ZI_ERR_ALIGN;
@@ -95,7 +96,7 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ZI_OK : ZI_ERR_CUDA;
@@ -156,25 +157,40 @@ enum KernelBit : unsigned {
 
 constexpr int kStages = 4;
 
-// sk.partials == nullptr: no split tail (a caller without workspace).
+template <int BN, int EPI, bool F8>
+struct GemmKernel {
+  static constexpr auto fn = gemm_bf16_tn_kernel<BN, kStages, EPI>;
+};
 template <int BN, int EPI>
-int run_gemm(DevInfo* dev, unsigned bit, int kind, const uint16_t* A, const uint16_t* B, int M, int N, int K,
+struct GemmKernel<BN, EPI, true> {
+  static constexpr auto fn = gemm_e4m3_tn_kernel<BN, kStages, EPI>;
+};
+
+// A [M, K] and B [N, K] are bf16, or e4m3 codes with F8 (then ep.a_scale [M] and
+// ep.b_scale [N] hold their per-row scales).  sk.partials == nullptr: no split
+// tail (a caller without workspace).
+template <int BN, int EPI, bool F8 = false>
+int run_gemm(DevInfo* dev, unsigned bit, int kind, const void* A, const void* B, int M, int N, int K,
              const EpiParams& ep, cudaStream_t st, SplitScratch sk = SplitScratch{nullptr, nullptr}) {
   using L = GemmSmem<BN, kStages>;
   static_assert(BN <= 256, "split partial slots hold 128 x 256 fp32");
+  constexpr int BK = F8 ? 128 : 64;  // elements per 128-byte smem row
+  constexpr uint64_t esz = F8 ? 1 : 2;
+  constexpr CUtensorMapDataType dt = F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (M <= 0) return ZI_OK;
-  if (K % 64 != 0 || N % BN != 0 || K <= 0 || N <= 0) return ZI_ERR_SHAPE;
+  if (K % BK != 0 || N % BN != 0 || K <= 0 || N <= 0) return ZI_ERR_SHAPE;
+  if (F8 && (!ep.a_scale || !ep.b_scale)) return ZI_ERR_ARG;
   CUtensorMap ta, tb;
-  ZI_TRY(make_map(&ta, A, uint64_t(K), uint64_t(M), uint64_t(K) * 2, 64, 128));
-  ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * 2, 64, BN));
-  auto kern = gemm_bf16_tn_kernel<BN, kStages, EPI>;
-  ZI_TRY(ensure_smem(dev, bit, kern, int(L::kBytes)));
+  ZI_TRY(make_map(&ta, A, uint64_t(K), uint64_t(M), uint64_t(K) * esz, BK, 128, dt));
+  ZI_TRY(make_map(&tb, B, uint64_t(K), uint64_t(N), uint64_t(K) * esz, BK, BN, dt));
+  auto kern = GemmKernel<BN, EPI, F8>::fn;
+  ZI_TRY(ensure_smem(dev, bit + (F8 ? 8u : 0u), kern, int(L::kBytes)));
   const int tiles = ((M + 127) / 128) * (N / BN);
-  const TailSched sched = make_tail_sched(tiles, dev->sms, K / 64, sk.partials != nullptr);
+  const TailSched sched = make_tail_sched(tiles, dev->sms, K / BK, sk.partials != nullptr);
   int grid = tiles < dev->sms ? tiles : dev->sms;
   if (sched.tail_items > grid) grid = sched.tail_items;  // fewer tiles than SMs, each cut along K
   prof_pre(st);
-  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, N, K, ep, sched, sk);
+  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, ep, sched, sk);
   return launched(kind, st);
 }
 
@@ -250,12 +266,13 @@ int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out
 
 // ---------------------------------------------------------------- row kernels
 
+// hq non-null: the output is e4m3 codes [rows][D] with per-row scales hs instead of bf16 h.
 template <typename TIn>
 int run_rms_mod(const TIn* x, int rows, int D, const uint16_t* gain, const float* scale, int scale_ld, RowMap map,
-                int row_off, float eps, uint16_t* h, cudaStream_t st) {
+                int row_off, float eps, uint16_t* h, cudaStream_t st, uint8_t* hq = nullptr, float* hs = nullptr) {
   if (rows <= 0) return ZI_OK;
   prof_pre(st);
-  rms_mod_kernel<TIn><<<rows, kRowThreads, 0, st>>>(x, D, gain, scale, scale_ld, map, row_off, eps, h);
+  rms_mod_kernel<TIn><<<rows, kRowThreads, 0, st>>>(x, D, gain, scale, scale_ld, map, row_off, eps, h, hq, hs);
   return launched(ZI_KERNEL_PRE_NORM, st);
 }
 
@@ -272,7 +289,7 @@ constexpr size_t kAlign = 1024;
 inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-  size_t mod, c, silu, hid, lens, pos, rope, x, h, qkv, att, o, u, tok, capn, split_cnt, split_part, total;
+  size_t mod, c, silu, hid, lens, pos, rope, x, h, hs, qkv, att, o, u, tok, capn, split_cnt, split_part, total;
 };
 
 Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int mod_cols) {
@@ -293,7 +310,8 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.pos = o; o = up(o + (model ? tab_rows * 3 * 4 : 0));
   w.rope = o; o = up(o + tab_rows * pairs * 8);
   w.x = o; o = up(o + (model ? rows * D * 4 : 0));
-  w.h = o; o = up(o + rows * D * 2);
+  w.h = o; o = up(o + rows * D * 2);  // bf16 h, or e4m3 codes (rows x D bytes) for e4m3 blocks
+  w.hs = o; o = up(o + rows * 4);      // per-row scales of e4m3 h
   w.qkv = o; o = up(o + rows * 3 * D * 2);
   w.att = o; o = up(o + rows * D * 2);
   w.o = o; o = up(o + rows * D * 2);
@@ -331,6 +349,9 @@ bool block_ptrs_ok(const zi_block_weights* w, bool need_mod) {
     if (!p) return false;
   if (need_mod && (!w->w_ada || !w->b_ada)) return false;
   if ((w->w_ada == nullptr) != (w->b_ada == nullptr)) return false;
+  // e4m3 projections: all four of w_qkv8, s_qkv, w13_8, s_13, or none
+  const int nf8 = (w->w_qkv8 != nullptr) + (w->s_qkv != nullptr) + (w->w13_8 != nullptr) + (w->s_13 != nullptr);
+  if (nf8 != 0 && nf8 != 4) return false;
   return true;
 }
 
@@ -339,6 +360,8 @@ bool block_align_ok(const zi_block_weights* w) {
   for (const void* p : ps)
     if (!aligned16(p)) return false;
   if (w->w_ada && !aligned16(w->w_ada)) return false;
+  if (w->w_qkv8 && (!aligned16(w->w_qkv8) || !aligned16(w->s_qkv) || !aligned16(w->w13_8) || !aligned16(w->s_13)))
+    return false;
   return true;
 }
 
@@ -348,7 +371,11 @@ struct NextNormSpec {
   const uint16_t* gain;
   const float* scale;  // [B][mod_ld] or null
   int next_rows;       // h written for local rows < next_rows
+  bool f8 = false;     // the next block takes e4m3 h (NEXT_RMS only)
 };
+
+// A block runs its QKV and FFN w1|w3 projections in e4m3 when it carries e4m3 weights.
+inline bool block_f8(const zi_block_weights* w) { return w && w->w_qkv8 != nullptr; }
 
 // One block over `rows` rows of the token buffer starting at global row `row_off`.
 // Pointers are local (row 0 = global row row_off).  h must already hold the
@@ -362,6 +389,8 @@ struct BlockCtx {
   float* x_in;
   float* x_out;
   uint16_t *h, *qkv, *att, *o, *u;
+  uint8_t* hq;  // the same buffer as h, as e4m3 codes (D bytes per row) for e4m3 blocks
+  float* hs;    // per-row scales of hq
   const float2* rope;
   const float* mod;  // this block's 4D modulation inside the per-batch vector, or null
   int mod_ld;
@@ -384,8 +413,16 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   eq.dim = D;
   eq.row_off = b.row_off;
   eq.map = b.map;
-  ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq, st,
-                                 b.split)));
+  const bool f8 = block_f8(b.w);
+  if (f8) {
+    eq.a_scale = b.hs;
+    eq.b_scale = b.w->s_qkv;
+    ZI_TRY((run_gemm<256, EPI_QKV, true>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.hq, b.w->w_qkv8, b.rows, 3 * D, D,
+                                         eq, st, b.split)));
+  } else {
+    ZI_TRY((run_gemm<256, EPI_QKV>(b.dev, BIT_GEMM_QKV, ZI_KERNEL_GEMM_QKV, b.h, b.w->w_qkv, b.rows, 3 * D, D, eq,
+                                   st, b.split)));
+  }
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len,
                        b.kv_len, st, b.split));
   ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D,
@@ -404,14 +441,24 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   pa.scale_ld = b.mod_ld;
   pa.next_rows = b.rows;
   pa.h = b.h;
+  pa.hq = f8 ? b.hq : nullptr;
+  pa.hs = f8 ? b.hs : nullptr;
   pa.map = b.map;
   pa.row_off = b.row_off;
   pa.D = D;
   pa.eps = eps;
   pa.eps_ln = b.cfg->final_eps;
   ZI_TRY(run_post(pa, b.rows, st));
-  ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp, D,
-                                    epi_plain(b.u, Fp), st, b.split)));
+  if (f8) {
+    EpiParams e13 = epi_plain(b.u, Fp);
+    e13.a_scale = b.hs;
+    e13.b_scale = b.w->s_13;
+    ZI_TRY((run_gemm<256, EPI_SWIGLU, true>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.hq, b.w->w13_8, b.rows,
+                                            2 * Fp, D, e13, st, b.split)));
+  } else {
+    ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp,
+                                      D, epi_plain(b.u, Fp), st, b.split)));
+  }
   ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp,
                                   epi_plain(b.o, D), st, b.split)));
   PostParams pf = pa;
@@ -422,6 +469,8 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   pf.g_next = next.gain;
   pf.scale = next.scale;
   pf.next_rows = next.next_rows;
+  pf.hq = (next.kind == NEXT_RMS && next.f8) ? b.hq : nullptr;
+  pf.hs = (next.kind == NEXT_RMS && next.f8) ? b.hs : nullptr;
   return run_post(pf, b.rows, st);
 }
 
@@ -611,6 +660,38 @@ int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m,
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+int zi_quantize_rows_e4m3(const void* d_x, int x_bf16, int rows, int cols, uint8_t* d_q, float* d_s,
+                          zi_stream_t stream) {
+  if (!d_x || !d_q || !d_s || rows < 0 || cols <= 0 || (x_bf16 != 0 && x_bf16 != 1)) return ZI_ERR_ARG;
+  if (cols % 4 || cols > kRowThreads * kRowMaxVec * 4) return ZI_ERR_SHAPE;
+  if (!aligned16(d_x) || !aligned16(d_q) || !aligned16(d_s)) return ZI_ERR_ALIGN;
+  DevInfo* dev;
+  ZI_TRY(current_device(&dev));
+  if (rows == 0) return ZI_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  prof_pre(st);
+  if (x_bf16)
+    quantize_rows_e4m3_kernel<uint16_t><<<rows, kRowThreads, 0, st>>>(static_cast<const uint16_t*>(d_x), cols, d_q, d_s);
+  else
+    quantize_rows_e4m3_kernel<float><<<rows, kRowThreads, 0, st>>>(static_cast<const float*>(d_x), cols, d_q, d_s);
+  return launched(ZI_KERNEL_QUANTIZE, st);
+}
+
+int zi_gemm_e4m3(const uint8_t* d_a, const float* d_sa, const uint8_t* d_b, const float* d_sb, uint16_t* d_c, int m,
+                 int n, int k, zi_stream_t stream) {
+  if (!d_a || !d_sa || !d_b || !d_sb || !d_c || m < 0 || n <= 0 || k <= 0) return ZI_ERR_ARG;
+  if (!aligned16(d_a) || !aligned16(d_b) || !aligned16(d_c) || !aligned16(d_sa) || !aligned16(d_sb))
+    return ZI_ERR_ALIGN;
+  if (k % 128 || n % 256) return ZI_ERR_SHAPE;
+  DevInfo* dev;
+  ZI_TRY(current_device(&dev));
+  EpiParams ep = epi_plain(d_c, n);
+  ep.a_scale = d_sa;
+  ep.b_scale = d_sb;
+  return run_gemm<256, EPI_BF16, true>(dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM, d_a, d_b, m, n, k, ep,
+                                       reinterpret_cast<cudaStream_t>(stream));
+}
+
 int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads, zi_stream_t stream) {
   if (!d_qkv || !d_out || batch <= 0 || seq <= 0 || heads <= 0) return ZI_ERR_ARG;
   if (!aligned16(d_qkv) || !aligned16(d_out)) return ZI_ERR_ALIGN;
@@ -680,6 +761,8 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.x_in = const_cast<float*>(d_x_in);
   b.x_out = d_x_out;
   b.h = reinterpret_cast<uint16_t*>(ws + L.h);
+  b.hq = ws + L.h;
+  b.hs = reinterpret_cast<float*>(ws + L.hs);
   b.qkv = reinterpret_cast<uint16_t*>(ws + L.qkv);
   b.att = reinterpret_cast<uint16_t*>(ws + L.att);
   b.o = reinterpret_cast<uint16_t*>(ws + L.o);
@@ -695,7 +778,9 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.kv_len = nullptr;
   b.split = SplitScratch{reinterpret_cast<float4*>(ws + L.split_part), reinterpret_cast<int*>(ws + L.split_cnt)};
   ZI_TRY(clear_split(b.split, st));
-  ZI_TRY(run_rms_mod<float>(d_x_in, rows, D, w->g_attn1, b.mod, b.mod_ld, b.map, 0, cfg->norm_eps, b.h, st));
+  const bool f8 = block_f8(w);
+  ZI_TRY(run_rms_mod<float>(d_x_in, rows, D, w->g_attn1, b.mod, b.mod_ld, b.map, 0, cfg->norm_eps, b.h, st,
+                            f8 ? b.hq : nullptr, f8 ? b.hs : nullptr));
   const NextNormSpec none{NEXT_NONE, nullptr, nullptr, 0};
   return run_block(b, none, st);
 }
@@ -741,6 +826,14 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     if (!block_ptrs_ok(&w->ctx[i], false) || w->ctx[i].w_ada || !block_align_ok(&w->ctx[i])) return ZI_ERR_ARG;
   for (int i = 0; i < cfg->n_main; ++i)
     if (!block_ptrs_ok(&w->main[i], true) || !block_align_ok(&w->main[i])) return ZI_ERR_ARG;
+  // every block in e4m3 or none (the blocks hand their normalised input h to each other)
+  const bool f8 = block_f8(&w->main[0]);
+  for (int i = 0; i < cfg->n_noise; ++i)
+    if (block_f8(&w->noise[i]) != f8) return ZI_ERR_ARG;
+  for (int i = 0; i < cfg->n_ctx; ++i)
+    if (block_f8(&w->ctx[i]) != f8) return ZI_ERR_ARG;
+  for (int i = 0; i < cfg->n_main; ++i)
+    if (block_f8(&w->main[i]) != f8) return ZI_ERR_ARG;
   if (!aligned16(w->x_emb_w) || !aligned16(w->cap_w) || !aligned16(w->final_w) || !aligned16(w->final_ada_w) ||
       !aligned16(w->x_emb_b) || !aligned16(w->cap_b) || !aligned16(w->cap_norm) || !aligned16(d_txt) ||
       !aligned16(d_latent) || !aligned16(d_out))
@@ -767,6 +860,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   float2* rope = reinterpret_cast<float2*>(ws + L.rope);
   float* x = reinterpret_cast<float*>(ws + L.x);
   uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  float* hs = reinterpret_cast<float*>(ws + L.hs);
   uint16_t* qkv = reinterpret_cast<uint16_t*>(ws + L.qkv);
   uint16_t* att = reinterpret_cast<uint16_t*>(ws + L.att);
   uint16_t* o = reinterpret_cast<uint16_t*>(ws + L.o);
@@ -888,6 +982,8 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     b.x_in = x + size_t(row_off) * D;
     b.x_out = b.x_in;
     b.h = h + size_t(row_off) * D;
+    b.hq = ws + L.h + size_t(row_off) * D;  // e4m3 rows are D bytes
+    b.hs = hs + row_off;
     b.qkv = qkv + size_t(row_off) * 3 * D;
     b.att = att + size_t(row_off) * D;
     b.o = o + size_t(row_off) * D;
@@ -899,7 +995,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     b.seg_len[1] = 1;
     return b;
   };
-  const NextNormSpec to_main0{NEXT_RMS, w->main[0].g_attn1, mod_of_main(0), 0};
+  const NextNormSpec to_main0{NEXT_RMS, w->main[0].g_attn1, mod_of_main(0), 0, f8};
 
   // noise refiners on the image rows (all keys are image tokens: no key mask)
   {
@@ -907,38 +1003,39 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     b.kv_len = nullptr;
     if (cfg->n_noise > 0) {
       ZI_TRY(run_rms_mod<float>(b.x_in, rows_img, D, w->noise[0].g_attn1, mod_of_noise(0), mod_ld, map, 0, eps,
-                                b.h, st));
+                                b.h, st, f8 ? b.hq : nullptr, b.hs));
       for (int i = 0; i < cfg->n_noise; ++i) {
         b.w = &w->noise[i];
         b.mod = mod_of_noise(i);
         NextNormSpec nx = to_main0;
-        if (i + 1 < cfg->n_noise) nx = NextNormSpec{NEXT_RMS, w->noise[i + 1].g_attn1, mod_of_noise(i + 1), 0};
+        if (i + 1 < cfg->n_noise) nx = NextNormSpec{NEXT_RMS, w->noise[i + 1].g_attn1, mod_of_noise(i + 1), 0, f8};
         nx.next_rows = rows_img;
         ZI_TRY(run_block(b, nx, st));
         ZI_TRY(trace());
       }
     } else {
       ZI_TRY(run_rms_mod<float>(b.x_in, rows_img, D, w->main[0].g_attn1, mod_of_main(0), mod_ld, map, 0, eps, b.h,
-                                st));
+                                st, f8 ? b.hq : nullptr, b.hs));
     }
   }
   // context refiners on the text rows (unmodulated)
   {
     BlockCtx b = segment_ctx(rows_img, rows_txt, s_txt);
     if (cfg->n_ctx > 0) {
-      ZI_TRY(run_rms_mod<float>(b.x_in, rows_txt, D, w->ctx[0].g_attn1, nullptr, 0, map, rows_img, eps, b.h, st));
+      ZI_TRY(run_rms_mod<float>(b.x_in, rows_txt, D, w->ctx[0].g_attn1, nullptr, 0, map, rows_img, eps, b.h, st,
+                                f8 ? b.hq : nullptr, b.hs));
       for (int i = 0; i < cfg->n_ctx; ++i) {
         b.w = &w->ctx[i];
         b.mod = nullptr;
         NextNormSpec nx = to_main0;
-        if (i + 1 < cfg->n_ctx) nx = NextNormSpec{NEXT_RMS, w->ctx[i + 1].g_attn1, nullptr, 0};
+        if (i + 1 < cfg->n_ctx) nx = NextNormSpec{NEXT_RMS, w->ctx[i + 1].g_attn1, nullptr, 0, f8};
         nx.next_rows = rows_txt;
         ZI_TRY(run_block(b, nx, st));
         ZI_TRY(trace());
       }
     } else {
       ZI_TRY(run_rms_mod<float>(b.x_in, rows_txt, D, w->main[0].g_attn1, mod_of_main(0), mod_ld, map, rows_img, eps,
-                                b.h, st));
+                                b.h, st, f8 ? b.hq : nullptr, b.hs));
     }
   }
   // main blocks on the joint sequence (two segments per batch element)
@@ -953,7 +1050,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
       b.w = &w->main[i];
       b.mod = mod_of_main(i);
       NextNormSpec nx{NEXT_LAYERNORM, nullptr, final_scale, rows_img};
-      if (i + 1 < cfg->n_main) nx = NextNormSpec{NEXT_RMS, w->main[i + 1].g_attn1, mod_of_main(i + 1), rows};
+      if (i + 1 < cfg->n_main) nx = NextNormSpec{NEXT_RMS, w->main[i + 1].g_attn1, mod_of_main(i + 1), rows, f8};
       ZI_TRY(run_block(b, nx, st));
       ZI_TRY(trace());
     }

@@ -67,9 +67,14 @@ TOP_KEYS = {
 
 
 class DeviceBlock:
-    """One block's weights in the library's layout (fused qkv, interleaved w13, padded w2)."""
+    """One block's weights in the library's layout (fused qkv, interleaved w13, padded w2).
 
-    def __init__(self, cfg: abi.ZiConfig, prefix: str, bits: Dict[str, Bits], modulated: bool, device):
+    fp8=True also stores e4m3 codes of the fused qkv and w13 with one scale per
+    output channel (zi_quantize_rows_e4m3); the block then runs those two
+    projections in e4m3."""
+
+    def __init__(self, cfg: abi.ZiConfig, prefix: str, bits: Dict[str, Bits], modulated: bool, device,
+                 fp8: bool = False):
         D, F = cfg.dim, cfg.ffn
         Fp = abi.ffn_padded(F)
         a = f"{prefix}.attention"
@@ -96,6 +101,10 @@ class DeviceBlock:
             self.t["w_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.weight"], device)
             self.t["b_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.bias"], device)
         self.modulated = modulated
+        if fp8:
+            for src, q, sc in (("w_qkv", "w_qkv8", "s_qkv"), ("w13", "w13_8", "s_13")):
+                self.t[q], self.t[sc] = quantize_rows_e4m3(self.t[src])
+        self.fp8 = fp8
         self.struct = abi.ZiBlockWeights(**{f: (self.t[f].data_ptr() if f in self.t else None)
                                             for f in abi.BLOCK_FIELDS})
 
@@ -106,19 +115,22 @@ class DeviceBlock:
 class DiT:
     """The S3-DiT transformer on one GPU, weights resident in HBM."""
 
-    def __init__(self, cfg: abi.ZiConfig, fetch: Callable[[Sequence[str]], Dict[str, Bits]], device="cuda"):
+    def __init__(self, cfg: abi.ZiConfig, fetch: Callable[[Sequence[str]], Dict[str, Bits]], device="cuda",
+                 fp8: bool = False):
         """fetch(keys) -> {key: bf16 bits} is called once per block and once for the rest,
-        so a 12 GB model never has to sit in host memory at once."""
+        so a 12 GB model never has to sit in host memory at once.  fp8=True runs every
+        block's QKV and FFN w1|w3 projections in e4m3 (see DeviceBlock)."""
         self.cfg = cfg
         self.device = torch.device(device)
         abi.lib()
         top = fetch(list(TOP_KEYS.values()))
         self.top = {f: upload_bits(top[k], self.device) for f, k in TOP_KEYS.items()}
+        self.fp8 = fp8
         self.noise = [DeviceBlock(cfg, f"noise_refiner.{i}", fetch(block_keys(f"noise_refiner.{i}", True)), True,
-                                  self.device) for i in range(cfg.n_noise)]
+                                  self.device, fp8) for i in range(cfg.n_noise)]
         self.ctx = [DeviceBlock(cfg, f"context_refiner.{i}", fetch(block_keys(f"context_refiner.{i}", False)),
-                                False, self.device) for i in range(cfg.n_ctx)]
-        self.main = [DeviceBlock(cfg, f"layers.{i}", fetch(block_keys(f"layers.{i}", True)), True, self.device)
+                                False, self.device, fp8) for i in range(cfg.n_ctx)]
+        self.main = [DeviceBlock(cfg, f"layers.{i}", fetch(block_keys(f"layers.{i}", True)), True, self.device, fp8)
                      for i in range(cfg.n_main)]
         self._noise_arr = (abi.ZiBlockWeights * max(1, len(self.noise)))(*[b.struct for b in self.noise])
         self._ctx_arr = (abi.ZiBlockWeights * max(1, len(self.ctx)))(*[b.struct for b in self.ctx])
@@ -305,6 +317,27 @@ def attention(qkv: torch.Tensor, batch: int, seq: int, heads: int,
         abi.call("zi_attention", _p(qkv), _p(out), batch, seq, heads, _stream())
     else:
         abi.call("zi_attention_varlen", _p(qkv), _p(out), batch, seq, heads, _p(kv_len), _stream())
+    return out
+
+
+def quantize_rows_e4m3(x: torch.Tensor):
+    """Per-row e4m3 codes (uint8, x's shape) and fp32 scales [rows] of a 2-D fp32 or bf16 tensor."""
+    assert x.dim() == 2 and x.is_contiguous() and x.dtype in (torch.float32, torch.bfloat16)
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(x.shape[0], dtype=torch.float32, device=x.device)
+    abi.call("zi_quantize_rows_e4m3", _p(x), 1 if x.dtype == torch.bfloat16 else 0, x.shape[0], x.shape[1], _p(q),
+             _p(sc), _stream())
+    return q, sc
+
+
+def gemm_e4m3(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """bf16 [M, N] = sa[m] sb[n] (a e4m3 [M, K]) (b e4m3 [N, K])^T."""
+    M, K = a.shape
+    N = b.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    abi.call("zi_gemm_e4m3", _p(a), _p(sa), _p(b), _p(sb), _p(out), M, N, K, _stream())
     return out
 
 
