@@ -44,7 +44,8 @@ struct EpiParams {
   void* out;
   int ldo;                 // row stride of `out` in elements
   const uint16_t* bias;    // bf16 [N] (EPI_F32_BIAS, EPI_UNPATCH)
-  const float2* rope;      // (cos, sin) [n_pos][head_dim / 2] (EPI_QKV)
+  const float2* rope;      // (cos, sin) [head_dim / 2][rope_n]: pair-major, so a warp's 32 rows
+  int rope_n;              // (consecutive positions) read one pair in one coalesced load (EPI_QKV)
   const uint16_t* g_q;     // bf16 [128] QK-RMSNorm gains (EPI_QKV)
   const uint16_t* g_k;
   float eps;
@@ -81,8 +82,10 @@ ZI_DEV void store_bf16x32(uint16_t* dst, const float* v) {
   }
 }
 
-// Epilogue of one tile of `width` columns (width <= BN, a multiple of 64)
-// starting at output column n0.
+// Epilogue of one half of a tile (`half` 0 or 1: two groups of 4 epilogue warps
+// share each tile), for the tile starting at output column n0.  Generic epilogues
+// take columns [half BN/2, (half + 1) BN/2); QKV one 128-wide head each; SwiGLU
+// the gate/up pairs [64 half, 64 half + 64).
 // acc[i] *= sa * b_scale[col + i] for 32 accumulator columns (e4m3 operands).
 ZI_DEV void scale_acc32(uint32_t* v, float sa, const float* b_scale, int col) {
   const float4* bs = reinterpret_cast<const float4*>(b_scale + col);
@@ -97,14 +100,15 @@ ZI_DEV void scale_acc32(uint32_t* v, float sa, const float* b_scale, int col) {
 }
 
 template <int EPI, int BN, bool F8>
-ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int width, const EpiParams& ep) {
+ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int half, const EpiParams& ep) {
+  constexpr int kChunks = BN / 64;  // 32-column chunks per half
   static_assert(!F8 || EPI == EPI_BF16 || EPI == EPI_QKV || EPI == EPI_SWIGLU, "e4m3 epilogues: bf16, QKV, SwiGLU");
   uint32_t v[32];
   float f[32];
   const float sa = (F8 && row_ok) ? __ldg(ep.a_scale + row) : 1.f;
   if constexpr (EPI == EPI_BF16 || EPI == EPI_F32_BIAS) {
 #pragma unroll 1
-    for (int c = 0; c < width / 32; ++c) {
+    for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
       tmem_ld32_sync(tbase + c * 32, v);
       if (row_ok) {
         const int col = n0 + c * 32;
@@ -139,7 +143,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
     uint16_t* orow = static_cast<uint16_t*>(ep.out) + size_t(row) * ep.ldo;
     if (region == 2) {
 #pragma unroll 1
-      for (int c = 0; c < width / 32; ++c) {
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         tmem_ld32_sync(tbase + c * 32, v);
         if (row_ok) {
           if constexpr (F8) scale_acc32(v, sa, ep.b_scale, n0 + c * 32);
@@ -152,9 +156,9 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
     }
     const uint16_t* g = region == 0 ? ep.g_q : ep.g_k;
     const int p = row_ok ? ep.map.tab(row + ep.row_off) : 0;
-    const float2* rp = ep.rope + size_t(p) * 64;
+    const float2* rp = ep.rope + p;  // pair j at rp[j * rope_n]
 #pragma unroll 1
-    for (int hh = 0; hh < width / 128; ++hh) {
+    for (int hh = half; hh < half + 1; ++hh) {  // one 128-wide head per half
       float ss = 0.f;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -172,12 +176,16 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
         tmem_ld32_sync(tbase + hh * 128 + c * 32, v);
         if (row_ok) {
           if constexpr (F8) scale_acc32(v, sa, ep.b_scale, n0 + hh * 128 + c * 32);
+          uint4 gw[4];  // the 32 gains of this chunk (the same for every row: broadcast loads)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) gw[k] = __ldg(reinterpret_cast<const uint4*>(g + c * 32) + k);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int d0 = c * 32 + 2 * i;
-            const float a = __uint_as_float(v[2 * i]) * r * bf16_to_f32(__ldg(g + d0));
-            const float b = __uint_as_float(v[2 * i + 1]) * r * bf16_to_f32(__ldg(g + d0 + 1));
-            const float2 cs = __ldg(rp + c * 16 + i);
+            const uint32_t gp = (i & 3) == 0 ? gw[i >> 2].x : (i & 3) == 1 ? gw[i >> 2].y
+                              : (i & 3) == 2 ? gw[i >> 2].z : gw[i >> 2].w;  // gains of dims 2i, 2i + 1
+            const float a = __uint_as_float(v[2 * i]) * r * __uint_as_float(gp << 16);
+            const float b = __uint_as_float(v[2 * i + 1]) * r * __uint_as_float(gp & 0xFFFF0000u);
+            const float2 cs = __ldg(rp + size_t(c * 16 + i) * ep.rope_n);
             f[2 * i] = a * cs.x - b * cs.y;
             f[2 * i + 1] = a * cs.y + b * cs.x;
           }
@@ -190,7 +198,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
     uint32_t u[32];
     uint16_t* orow = static_cast<uint16_t*>(ep.out) + size_t(row) * ep.ldo + n0 / 2;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {
       tmem_ld32(tbase + c * 32, v);
       tmem_ld32(tbase + 128 + c * 32, u);
       tmem_wait_ld();
@@ -216,7 +224,7 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
     const int b = gr / ep.s_img, t = gr % ep.s_img;
     const int ty = t / ep.grid_w, tx = t % ep.grid_w;
 #pragma unroll 1
-    for (int c = 0; c < width / 32; ++c) {
+    for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
       tmem_ld32_sync(tbase + c * 32, v);
       if (row_ok) {
 #pragma unroll 4
@@ -243,6 +251,8 @@ ZI_DEV void gemm_epilogue(uint32_t tbase, int row, bool row_ok, int n0, int widt
 // (the same order whichever piece finishes, so results are deterministic) and
 // runs the fused epilogue.  No CTA waits for another.
 constexpr int kMaxSplit = 4;
+constexpr int kEpiWarps = 8;                        // two groups of 4 (each covers all 128 TMEM lanes)
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;   // + the TMA and MMA warps
 constexpr int kMinSplitKb = 4;
 constexpr int kSplitSlots = 160;  // partial slots (>= G); counters likewise
 
@@ -340,10 +350,10 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * kEpiWarps);
     }
     mbar_init(drain, 1);
-    mbar_init(ebar, 128);
+    mbar_init(ebar, 32 * kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -443,11 +453,12 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
       }
     }
   } else {
-    const int q = warp & 3;  // this warp's TMEM lane quarter
+    const int q = warp & 3;             // this warp's TMEM lane quarter
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row_in_tile = q * 32 + lane;
     int local = 0;
     uint32_t ephase = 0;
-    auto epi_sync = [&]() -> bool {  // the 128 epilogue threads meet (bounded wait)
+    auto epi_sync = [&]() -> bool {  // the epilogue threads meet (bounded wait)
       mbar_arrive(ebar);
       const bool r = mbar_wait(ebar, ephase, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE);
       ephase ^= 1u;
@@ -468,7 +479,7 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
         // A piece of a split tile: publish the partial, then finish only if last.
         const int slot0 = blockIdx.x - wi.piece;  // slot of piece 0 of this tile
         float4* mine = sk.partials + size_t(blockIdx.x) * (32 * BN) + row_in_tile;
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
           uint32_t v[32];
           tmem_ld32_sync(tb + c * 32, v);
 #pragma unroll
@@ -490,46 +501,49 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
         finish = *last_flag != 0;
         if (finish) {
           __threadfence();
-          for (int c = 0; c < BN / 32; ++c) {
-            // Every other piece's 32 columns are loaded before any is used, so up to
-            // (kMaxSplit - 1) x 8 loads are in flight instead of one at a time.
-            float4 pp[kMaxSplit][8];
-#pragma unroll
-            for (int j = 0; j < kMaxSplit; ++j) {
-              const bool need = j < sched.tail_s && j != wi.piece;
-              const float4* src = sk.partials + size_t(slot0 + j) * (32 * BN) + size_t(c * 8) * 128 + row_in_tile;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) pp[j][k] = need ? __ldcg(src + size_t(k) * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+          for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+            // Sum the pieces in piece order 0, 1, ..., s - 1 whichever piece finishes;
+            // each other piece's 8 loads are issued together.
             uint32_t v[32];
             tmem_ld32_sync(tb + c * 32, v);
+            float4 tot[8];
+            for (int j = 0; j < sched.tail_s; ++j) {
+              float4 pj[8];
+              if (j == wi.piece) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float4 own = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                             __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
-              // sum in piece order 0, 1, ..., s - 1 whichever piece finishes
-              float4 tot = wi.piece == 0 ? own : pp[0][k];
+                for (int k = 0; k < 8; ++k)
+                  pj[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                      __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+              } else {
+                const float4* src = sk.partials + size_t(slot0 + j) * (32 * BN) + size_t(c * 8) * 128 + row_in_tile;
 #pragma unroll
-              for (int j = 1; j < kMaxSplit; ++j) {
-                if (j < sched.tail_s) {
-                  const float4 pj = j == wi.piece ? own : pp[j][k];
-                  tot.x += pj.x;
-                  tot.y += pj.y;
-                  tot.z += pj.z;
-                  tot.w += pj.w;
+                for (int k = 0; k < 8; ++k) pj[k] = __ldcg(src + size_t(k) * 128);
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                if (j == 0) {
+                  tot[k] = pj[k];
+                } else {
+                  tot[k].x += pj[k].x;
+                  tot[k].y += pj[k].y;
+                  tot[k].z += pj[k].z;
+                  tot[k].w += pj[k].w;
                 }
               }
-              v[4 * k] = __float_as_uint(tot.x);
-              v[4 * k + 1] = __float_as_uint(tot.y);
-              v[4 * k + 2] = __float_as_uint(tot.z);
-              v[4 * k + 3] = __float_as_uint(tot.w);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              v[4 * k] = __float_as_uint(tot[k].x);
+              v[4 * k + 1] = __float_as_uint(tot[k].y);
+              v[4 * k + 2] = __float_as_uint(tot[k].z);
+              v[4 * k + 3] = __float_as_uint(tot[k].w);
             }
             tmem_st32(tb + c * 32, v);
           }
           tmem_wait_st();
         }
       }
-      if (finish) gemm_epilogue<EPI, BN, F8>(tb, row, row < M, n0, BN, ep);
+      if (finish) gemm_epilogue<EPI, BN, F8>(tb, row, row < M, n0, half, ep);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -543,14 +557,14 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
 }
 
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
                         EpiParams ep, TailSched sched, SplitScratch sk) {
   gemm_tn_body<BN, STAGES, EPI, false>(tmA, tmB, M, ep, sched, sk);
 }
 
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_e4m3_tn_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
                         EpiParams ep, TailSched sched, SplitScratch sk) {
   gemm_tn_body<BN, STAGES, EPI, true>(tmA, tmB, M, ep, sched, sk);

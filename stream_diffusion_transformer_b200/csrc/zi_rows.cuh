@@ -330,8 +330,9 @@ __global__ void text_pad_kernel(float* __restrict__ x_txt, int s_txt, int D, con
 // (cos, sin) of pos[axis] * theta^(-2j/d_axis) for every token and rotation
 // pair; pairs [0, a0/2) use axis 0, the next a1/2 axis 1, the last a2/2 axis 2.
 // Angles are formed in fp64 and rounded to fp32 once.
+// out[t][j] (pos_major) or out[j][t] (pair-major, the layout the QKV epilogue reads).
 __global__ void rope_table_kernel(const int* __restrict__ pos, int n, int a0, int a1, int a2, double theta,
-                                  float2* __restrict__ out) {
+                                  float2* __restrict__ out, int pos_major) {
   const int pairs = (a0 + a1 + a2) / 2;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n * pairs) return;
@@ -348,7 +349,7 @@ __global__ void rope_table_kernel(const int* __restrict__ pos, int n, int a0, in
   const double ang = double(pos[3 * t + axis]) * omega;
   double s, c;
   sincos(ang, &s, &c);
-  out[idx] = make_float2(float(c), float(s));
+  out[pos_major ? idx : size_t(j) * n + t] = make_float2(float(c), float(s));
 }
 
 // Timestep conditioning, step 1: hid[b] = SiLU(W1 e + b1) with

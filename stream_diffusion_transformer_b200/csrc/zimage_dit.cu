@@ -190,7 +190,7 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const void* A, const void* B,
   int grid = tiles < dev->sms ? tiles : dev->sms;
   if (sched.tail_items > grid) grid = sched.tail_items;  // fewer tiles than SMs, each cut along K
   prof_pre(st);
-  kern<<<grid, 192, L::kBytes, st>>>(ta, tb, M, ep, sched, sk);
+  kern<<<grid, kGemmThreads, L::kBytes, st>>>(ta, tb, M, ep, sched, sk);
   return launched(kind, st);
 }
 
@@ -356,7 +356,7 @@ bool block_ptrs_ok(const zi_block_weights* w, bool need_mod) {
 }
 
 bool block_align_ok(const zi_block_weights* w) {
-  const void* ps[] = {w->w_qkv, w->w_out, w->w13, w->w2, w->g_attn1, w->g_attn2, w->g_ffn1, w->g_ffn2};
+  const void* ps[] = {w->w_qkv, w->w_out, w->w13, w->w2, w->g_attn1, w->g_attn2, w->g_ffn1, w->g_ffn2, w->g_q, w->g_k};
   for (const void* p : ps)
     if (!aligned16(p)) return false;
   if (w->w_ada && !aligned16(w->w_ada)) return false;
@@ -391,7 +391,8 @@ struct BlockCtx {
   uint16_t *h, *qkv, *att, *o, *u;
   uint8_t* hq;  // the same buffer as h, as e4m3 codes (D bytes per row) for e4m3 blocks
   float* hs;    // per-row scales of hq
-  const float2* rope;
+  const float2* rope;  // pair-major [head_dim / 2][rope_n]
+  int rope_n;
   const float* mod;  // this block's 4D modulation inside the per-batch vector, or null
   int mod_ld;
   int nseg;
@@ -407,6 +408,7 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   // QKV projection with QK-RMSNorm + RoPE epilogue
   EpiParams eq = epi_plain(b.qkv, 3 * D);
   eq.rope = b.rope;
+  eq.rope_n = b.rope_n;
   eq.g_q = b.w->g_q;
   eq.g_k = b.w->g_k;
   eq.eps = eps;
@@ -484,12 +486,14 @@ int run_ada(const AdaSegs& segs, const float* c, const float* silu_c, int batch,
   return launched(ZI_KERNEL_ADALN, st);
 }
 
-int run_rope(const zi_config& cfg, const int32_t* pos, int n, float2* out, cudaStream_t st) {
+// pos_major: out [n][pairs] (the zi_rope_table layout); else [pairs][n] for the QKV epilogue.
+int run_rope(const zi_config& cfg, const int32_t* pos, int n, float2* out, cudaStream_t st, bool pos_major) {
   const int pairs = cfg.head_dim / 2;
   const int total = n * pairs;
   prof_pre(st);
   rope_table_kernel<<<(total + 255) / 256, 256, 0, st>>>(pos, n, cfg.rope_axes[0], cfg.rope_axes[1],
-                                                           cfg.rope_axes[2], double(cfg.rope_theta), out);
+                                                           cfg.rope_axes[2], double(cfg.rope_theta), out,
+                                                           pos_major ? 1 : 0);
   return launched(ZI_KERNEL_ROPE, st);
 }
 
@@ -647,7 +651,8 @@ int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, float* d_co
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
   if (n == 0) return ZI_OK;
-  return run_rope(*cfg, d_pos, n, reinterpret_cast<float2*>(d_cos_sin), reinterpret_cast<cudaStream_t>(stream));
+  return run_rope(*cfg, d_pos, n, reinterpret_cast<float2*>(d_cos_sin), reinterpret_cast<cudaStream_t>(stream),
+                  true);
 }
 
 int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k, zi_stream_t stream) {
@@ -748,7 +753,7 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
     segs.dim = D;
     ZI_TRY(run_ada(segs, d_c, d_c, batch, 4 * D, mod, st));
   }
-  ZI_TRY(run_rope(*cfg, d_pos, seq, rope, st));
+  ZI_TRY(run_rope(*cfg, d_pos, seq, rope, st, false));
 
   BlockCtx b;
   b.dev = dev;
@@ -768,6 +773,7 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.o = reinterpret_cast<uint16_t*>(ws + L.o);
   b.u = reinterpret_cast<uint16_t*>(ws + L.u);
   b.rope = rope;
+  b.rope_n = seq;
   b.mod = modulated ? mod : nullptr;
   b.mod_ld = 4 * D;
   b.nseg = 1;
@@ -925,7 +931,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     prof_pre(st);
     positions_kernel<<<(S + 255) / 256, 256, 0, st>>>(s_txt, gh, gw, pos);
     ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
-    ZI_TRY(run_rope(*cfg, pos, S, rope, st));
+    ZI_TRY(run_rope(*cfg, pos, S, rope, st, false));
   } else {
     for (int b0 = 0; b0 < batch; b0 += kLenChunk) {
       LenChunk ch;
@@ -940,7 +946,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     prof_pre(st);
     positions_varlen_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(s_txt, gh, gw, lens, batch, pos);
     ZI_TRY(launched(ZI_KERNEL_POSITIONS, st));
-    ZI_TRY(run_rope(*cfg, pos, rows, rope, st));
+    ZI_TRY(run_rope(*cfg, pos, rows, rope, st, false));
   }
 
   // embedders: image rows [0, rows_img), text rows [rows_img, rows)
@@ -971,6 +977,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   base.batch = batch;
   base.map = map;
   base.rope = rope;
+  base.rope_n = h_txt_len ? rows : S;  // one table per element with text lengths
   base.mod_ld = mod_ld;
   base.kv_len = lens;
   base.split = split;
