@@ -59,8 +59,9 @@ constexpr int kRegsSoftmax = 216;  // 2 x 128 x 216 + 128 x 56 = 62464 <= 384 x 
 constexpr int kRegsOther = 56;
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile (two 64-column halves)
 constexpr uint32_t kHalf = kTile / 2;
-constexpr uint32_t kQ0 = 0, kK0 = 2 * kTile, kV0 = 4 * kTile;
-constexpr uint32_t kBar = 6 * kTile;
+constexpr int kKSlots = 3, kVSlots = 2;  // K ring one deeper than V (smem holds 7 tiles)
+constexpr uint32_t kQ0 = 0, kK0 = 2 * kTile, kV0 = kK0 + kKSlots * kTile;
+constexpr uint32_t kBar = kV0 + kVSlots * kTile;
 constexpr uint32_t kSmemBytes = kBar + 256 + 1024;
 constexpr uint32_t kColS = 0, kColO = 256;  // S_t at kColS + 128 t, O_t at kColO + 128 t
 constexpr int kMaxSplit = 4;
@@ -165,16 +166,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2 tiles]
-  uint64_t* p_full = bars + 11;  // [2 tiles]
-  uint64_t* pv_done = bars + 13; // [2 tiles]
-  uint64_t* drain = bars + 15;
-  uint64_t* fin_bar = bars + 16;  // the softmax threads' meeting point (split pieces)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* k_full = bars + 1;    // [kKSlots]
+  uint64_t* k_empty = bars + 4;   // [kKSlots]
+  uint64_t* v_full = bars + 7;    // [kVSlots]
+  uint64_t* v_empty = bars + 9;   // [kVSlots]
+  uint64_t* s_full = bars + 11;   // [2 tiles]
+  uint64_t* p_full = bars + 13;   // [2 tiles]
+  uint64_t* pv_done = bars + 15;  // [2 tiles]
+  uint64_t* drain = bars + 17;
+  uint64_t* fin_bar = bars + 18;  // the softmax threads' meeting point (split pieces)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* fin_flag = abort_flag + 1;
 
@@ -198,11 +199,15 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKSlots; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
       mbar_init(&pv_done[i], 1);
@@ -248,11 +253,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       uint64_t* emptyb = kq ? k_empty : v_empty;
       const uint32_t base = kq ? kK0 : kV0;
       const int col = kq ? colk : colv;
+      const int nslots = kq ? kKSlots : kVSlots;
       uint32_t issued = 0;
       bool ok = true;
       for (int j = 0; j < nj; ++j) {
-        const int bi = j & 1;
-        const uint32_t r = uint32_t(j) >> 1;
+        const int bi = j % nslots;
+        const uint32_t r = uint32_t(j / nslots);
         int kv0, kvn;
         attn_tile_rows(p, b, j0 + j, last_keys, kv0, kvn);
         if (!mbar_wait(&emptyb[bi], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) { ok = false; break; }
@@ -264,8 +270,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       if (!ok) {
         volatile int never = 0;
         if (kq) mbar_wait(q_full, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
-        for (uint32_t j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-          mbar_wait(&fullb[j & 1], (j >> 1) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
+        for (uint32_t j = (issued > uint32_t(nslots) ? issued - nslots : 0); j < issued; ++j)
+          mbar_wait(&fullb[j % nslots], (j / nslots) & 1u, &never, ZI_DEVERR_TIMEOUT_DRAIN);
       }
     }
    } else if (warp == 9) {
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       // S_t(j) = Q_t K_j^T into S_t
       auto issue_s = [&](int t, int j) {
         const uint32_t q_addr = smem_u32(smem + kQ0 + t * kTile);
-        const uint32_t k_addr = smem_u32(smem + kK0 + (j & 1) * kTile);
+        const uint32_t k_addr = smem_u32(smem + kK0 + (j % kKSlots) * kTile);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint64_t ad = smem_desc_sw128(q_addr + (k >> 2) * kHalf + (k & 3) * 32, 16);
@@ -302,7 +308,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         return true;
       };
       auto wait_k = [&](int j) {
-        return mbar_wait(&k_full[j & 1], (uint32_t(j) >> 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA);
+        return mbar_wait(&k_full[j % kKSlots], uint32_t(j / kKSlots) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA);
       };
       auto wait_v = [&](int j) {
         return mbar_wait(&v_full[j & 1], (uint32_t(j) >> 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA);
@@ -328,7 +334,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tc_commit(&v_empty[j & 1]);
         if (more) {
           if (ntile > 1) issue_s(1, j + 1);
-          tc_commit(&k_empty[(j + 1) & 1]);
+          tc_commit(&k_empty[(j + 1) % kKSlots]);
           if (!wait_v(j + 1) || !issue_pv(0, j + 1)) { ok = false; break; }
         }
       }
