@@ -15,8 +15,10 @@ module states one (a reading, shared with the GPU path):
     NaN; the largest finite magnitude is 448 (S.1111.110).  Rounding to nearest,
     ties to the even code; magnitudes beyond 448 saturate to 448.
   * which projections: the two whose input is a whole-row RMSNorm output, the
-    fused QKV projection and the FFN w1|w3 projection.  The attention output
-    projection, FFN w2, the embedders, adaLN and the final layer stay bf16.
+    fused QKV projection and the FFN w1|w3 projection; optionally (all=True)
+    also the attention output projection and FFN w2, whose inputs (attention
+    output, SwiGLU output) are quantised per row the same way.  The embedders,
+    adaLN and the final layer stay bf16.
   * scales: one per row of each operand.  Activations h [M, K]: s_a[m] =
     amax_m / 448, codes = e4m3(h[m, :] * (448 / amax_m)).  Weights [N, K]: the
     same per output channel.  A row of zeros gets scale 1 and zero codes.
@@ -101,8 +103,10 @@ def fp8_linear(h: np.ndarray, w: np.ndarray) -> np.ndarray:
 
 
 def block_forward(x: np.ndarray, W: ref.Weights, prefix: str, d, angles: np.ndarray,
-                  c: Optional[np.ndarray] = None, key_valid: Optional[np.ndarray] = None) -> np.ndarray:
-    """The block of zimage_ref.block_forward with the QKV and FFN w1|w3 projections in e4m3.
+                  c: Optional[np.ndarray] = None, key_valid: Optional[np.ndarray] = None,
+                  all: bool = False) -> np.ndarray:
+    """The block of zimage_ref.block_forward with the QKV and FFN w1|w3 projections in e4m3
+    (all=True: the output projection and FFN w2 as well).
 
     h is quantised once per row and shared by q, k and v (one fused projection);
     every weight row (output channel) has its own scale."""
@@ -121,7 +125,7 @@ def block_forward(x: np.ndarray, W: ref.Weights, prefix: str, d, angles: np.ndar
     q = ref.apply_rope(ref.rms_norm(q, W(f"{a}.norm_q.weight")), angles)
     k = ref.apply_rope(ref.rms_norm(k, W(f"{a}.norm_k.weight")), angles)
     att = ref.attention(q, k, v, key_valid).reshape(S, D)
-    o = ref.linear(att, W(f"{a}.to_out.weight"))
+    o = fp8_linear(att, W(f"{a}.to_out.weight")) if all else ref.linear(att, W(f"{a}.to_out.weight"))
     x1 = x + gate_msa * ref.rms_norm(o, W(f"{prefix}.attention_norm2.weight"))
     h2 = ref.rms_norm(x1, W(f"{prefix}.ffn_norm1.weight")) * (1.0 + scale_mlp)
     ff = f"{prefix}.feed_forward"
@@ -129,12 +133,14 @@ def block_forward(x: np.ndarray, W: ref.Weights, prefix: str, d, angles: np.ndar
     g13 = fp8_linear(h2, w13)
     F = d.ffn
     u = ref.silu(g13[:, :F]) * g13[:, F:]
-    f = ref.linear(u, W(f"{ff}.w2.weight"))
+    f = fp8_linear(u, W(f"{ff}.w2.weight")) if all else ref.linear(u, W(f"{ff}.w2.weight"))
     return x1 + gate_mlp * ref.rms_norm(f, W(f"{prefix}.ffn_norm2.weight"))
 
 
-def model_forward(latent: np.ndarray, t: np.ndarray, txt: np.ndarray, W: ref.Weights, d) -> np.ndarray:
-    """zimage_ref.model_forward with every block's QKV and FFN w1|w3 projections in e4m3."""
+def model_forward(latent: np.ndarray, t: np.ndarray, txt: np.ndarray, W: ref.Weights, d,
+                  all: bool = False) -> np.ndarray:
+    """zimage_ref.model_forward with every block's QKV and FFN w1|w3 projections in e4m3
+    (all=True: every block projection)."""
     B, C, Hl, Wl = latent.shape
     p = d.patch
     gh, gw = Hl // p, Wl // p
@@ -149,12 +155,12 @@ def model_forward(latent: np.ndarray, t: np.ndarray, txt: np.ndarray, W: ref.Wei
         xi = ref.linear(tokens[b], W("x_embedder.weight"), W("x_embedder.bias"))
         xt = ref.embed_text(np.asarray(txt[b], dtype=W.dtype), W)
         for i in range(d.n_noise):
-            xi = block_forward(xi, W, f"noise_refiner.{i}", d, ang[:s_img], c)
+            xi = block_forward(xi, W, f"noise_refiner.{i}", d, ang[:s_img], c, all=all)
         for i in range(d.n_ctx):
-            xt = block_forward(xt, W, f"context_refiner.{i}", d, ang[s_img:], None)
+            xt = block_forward(xt, W, f"context_refiner.{i}", d, ang[s_img:], None, all=all)
         x = np.concatenate([xi, xt], axis=0)
         for i in range(d.n_main):
-            x = block_forward(x, W, f"layers.{i}", d, ang, c)
+            x = block_forward(x, W, f"layers.{i}", d, ang, c, all=all)
         y = ref.final_layer(x[:s_img], W, c)
         outs.append(ref.unpatchify(y[None], C, Hl, Wl, p)[0])
     return np.stack(outs, axis=0)

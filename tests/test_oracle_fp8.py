@@ -93,3 +93,19 @@ def test_fp8_block_tracks_the_bf16_block():
     y8 = f8.block_forward(x, W, "layers.0", d, ang, c)
     rel = np.linalg.norm((y8 - x) - (y16 - x)) / np.linalg.norm(y16 - x)
     assert 1e-4 < rel < 0.1
+
+
+def test_all_projection_block_moves_further_from_bf16():
+    """all=True also quantises the output projection and FFN w2: the block's update moves
+    further from the bf16 block than with two e4m3 projections, and stays within 20%."""
+    d = zi.TINY_R
+    bits = zi.make_weights(d, seed=5)
+    W = ref.Weights(bits)
+    x = zi.make_stream(d, 1, 24, seed=5)[0].astype(np.float64)
+    c = zi.make_cond(d, 1, seed=5)[0].astype(np.float64)
+    ang = ref.rope_angles(ref.position_ids(8, 4, 4), d.rope_axes)
+    y16 = ref.block_forward(x, W, "layers.0", d, ang, c)
+    y8 = f8.block_forward(x, W, "layers.0", d, ang, c)
+    y8a = f8.block_forward(x, W, "layers.0", d, ang, c, all=True)
+    e = lambda y: np.linalg.norm((y - x) - (y16 - x)) / np.linalg.norm(y16 - x)
+    assert 0 < e(y8) < e(y8a) < 0.2
