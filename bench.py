@@ -516,7 +516,7 @@ def run_cfg_workload(args):
         step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(0) as clocks, abi.Profile(capacity=300 * args.steps + 16) as prof:
+    with ClockSampler(0) as clocks, abi.Profile(capacity=400 * args.steps + 16) as prof:
         e0.record()
         for _ in range(args.steps):
             step()
@@ -533,7 +533,7 @@ def run_cfg_workload(args):
                       "clocks": clocks.summary()}), flush=True)
 
 
-def run_fp8_workload(args):
+def run_fp8_workload(args, mode=True):
     """The metric's forward (4,128 tokens at 1024x1024, batch 1) with every block's QKV
     and FFN w1|w3 projections in e4m3 (per-row scales, tcgen05 kind::f8f6f4); the other
     steps stay as in the bf16 forward.  FLOPs are counted as for the bf16 forward."""
@@ -544,7 +544,7 @@ def run_fp8_workload(args):
     d = zi.FULL
     threads = max(1, min(32, (os.cpu_count() or 8)))
     dit = model.DiT(model.make_config(d), lambda keys: zi.make_weights(d, seed=SEED, keys=keys, threads=threads),
-                    fp8=True)
+                    fp8=mode)
     lat = torch.from_numpy(zi.make_latent(d, 1, LAT_H, LAT_W, seed=SEED)).cuda()
     txt = torch.from_numpy(zi.make_text(d, 1, S_TXT, seed=SEED).view(np.int16)).cuda().view(torch.bfloat16)
     tt = torch.full((1,), T_VALUE, dtype=torch.float32, device="cuda")
@@ -553,7 +553,7 @@ def run_fp8_workload(args):
         dit.forward(lat, tt, txt, out)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(0) as clocks, abi.Profile(capacity=300 * args.steps + 16) as prof:
+    with ClockSampler(0) as clocks, abi.Profile(capacity=400 * args.steps + 16) as prof:
         e0.record()
         for _ in range(args.steps):
             dit.forward(lat, tt, txt, out)
@@ -567,7 +567,10 @@ def run_fp8_workload(args):
     peak_f8 = 2.0 * float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))  # e4m3 = 2x bf16 (nominal ratio)
     per_step = len(prof.kinds) // args.steps
     roof = {}
-    for kind, kfl in (("gemm_qkv_qknorm_rope", 6.0 * S * d.dim ** 2), ("gemm_ffn_up_swiglu", 4.0 * S * d.dim * d.ffn)):
+    kinds = [("gemm_qkv_qknorm_rope", 6.0 * S * d.dim ** 2), ("gemm_ffn_up_swiglu", 4.0 * S * d.dim * d.ffn)]
+    if mode == "all":
+        kinds += [("gemm_out_proj", 2.0 * S * d.dim ** 2), ("gemm_ffn_down", 2.0 * S * d.dim * d.ffn)]
+    for kind, kfl in kinds:
         ms_k = []
         for sidx in range(args.steps):
             seq = [m for k, m in zip(prof.kinds[sidx * per_step:(sidx + 1) * per_step],
@@ -578,9 +581,11 @@ def run_fp8_workload(args):
                       "frac": kfl / (m * 1e-3) / 1e12 / peak_f8,
                       "peak_source": f"{peak_src} bf16 sustained x 2 (nominal e4m3 / bf16 ratio)"}
     by = {k: {"launches": v[0], "ms": round(v[1] / args.steps, 3)} for k, v in prof.by_kernel().items()}
-    print(json.dumps({"workload": f"e4m3 QKV + FFN-up projections, 1024x1024, {s_img} + {S_TXT} tokens, batch 1",
+    what = "every block projection" if mode == "all" else "QKV + FFN-up projections"
+    print(json.dumps({"workload": f"e4m3 {what}, 1024x1024, {s_img} + {S_TXT} tokens, batch 1",
                       "ms_per_step": ms, "value": fl / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                      "dtype": "e4m3 (QKV, FFN w1|w3) + bf16", "flops_per_step": fl, "steps": args.steps,
+                      "dtype": "e4m3 (all block projections) + bf16" if mode == "all" else "e4m3 (QKV, FFN w1|w3) + bf16",
+                      "flops_per_step": fl, "steps": args.steps,
                       "warmup": args.warmup, "kernel_rooflines": roof, "kernels_ms_per_step": by,
                       "finite": bool(torch.isfinite(out).all().item()), "device_status": abi.device_status(),
                       "clocks": clocks.summary()}), flush=True)
@@ -593,7 +598,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8"], default="forward",
+    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8", "fp8all"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
                          "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens; "
                          "cfg: one guidance step at 2048x2048, batch 2 x 16,896 tokens")
@@ -607,8 +612,8 @@ def main():
     if args.workload == "cfg":
         run_cfg_workload(args)
         return
-    if args.workload == "fp8":
-        run_fp8_workload(args)
+    if args.workload in ("fp8", "fp8all"):
+        run_fp8_workload(args, "all" if args.workload == "fp8all" else True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

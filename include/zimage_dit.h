@@ -115,6 +115,13 @@ typedef struct zi_block_weights {
   const float* s_qkv;      /* [3D] ... these (zi_quantize_rows_e4m3 of w_qkv) */
   const uint8_t* w13_8;    /* [2Fp, D] e4m3 codes of w13 */
   const float* s_13;       /* [2Fp] */
+  /* Optional, with the four above (all four, or all NULL): the output projection
+   * and FFN w2 in e4m3 too.  The attention output and the SwiGLU output are then
+   * quantised per row (the same recipe) by an extra pass before each GEMM. */
+  const uint8_t* w_out8;   /* [D, D] e4m3 codes of w_out */
+  const float* s_out;      /* [D] */
+  const uint8_t* w2_8;     /* [D, Fp] e4m3 codes of w2 (zero columns F..Fp) */
+  const float* s_2;        /* [D] */
 } zi_block_weights;
 
 /* Weights of the whole transformer.  The block arrays are HOST arrays (of
@@ -309,7 +316,7 @@ ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c,
  *   zeros gets s = 1 and zero codes.  The same recipe the norms use for e4m3 blocks.
  *   d_x   [rows, cols] fp32 (x_bf16 = 0) or bf16 (x_bf16 = 1), contiguous
  *   d_q   [rows, cols] uint8 codes;  d_s [rows] fp32 scales
- * cols % 4 == 0 and cols <= 4096 (ZI_ERR_SHAPE otherwise); 16-byte aligned pointers.
+ * cols % 4 == 0 and cols <= 16384 (ZI_ERR_SHAPE otherwise); 16-byte aligned pointers.
  * Weights for e4m3 blocks are made with it (rows = output channels). */
 ZI_API int zi_quantize_rows_e4m3(const void* d_x, int x_bf16, int rows, int cols, uint8_t* d_q, float* d_s,
                                  zi_stream_t stream);

@@ -34,7 +34,7 @@ class ZiConfig(ctypes.Structure):
 
 
 BLOCK_FIELDS = ("w_qkv", "w_out", "w13", "w2", "g_attn1", "g_attn2", "g_ffn1", "g_ffn2", "g_q", "g_k",
-                "w_ada", "b_ada", "w_qkv8", "s_qkv", "w13_8", "s_13")
+                "w_ada", "b_ada", "w_qkv8", "s_qkv", "w13_8", "s_13", "w_out8", "s_out", "w2_8", "s_2")
 
 
 class ZiBlockWeights(ctypes.Structure):

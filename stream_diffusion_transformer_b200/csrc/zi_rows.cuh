@@ -38,11 +38,12 @@ ZI_DEV float block_max(float v, float* red) {
 // Stores a row held by the CTA (y[k] for vector i = threadIdx.x + k * kRowThreads <
 // nvec) as e4m3 codes with one fp32 scale: amax / 448, codes of y * (448 / amax)
 // (round to nearest even, saturating); an all-zero row gets scale 1 and zero codes.
-// Every thread of the CTA must call it.
+// Every thread of the CTA must call it.  MAXVEC: float4 per thread the row may need.
+template <int MAXVEC = kRowMaxVec>
 ZI_DEV void store_row_e4m3(const float4* y, int nvec, float* red, uint8_t* q, float* scale) {
   float m = 0.f;
 #pragma unroll
-  for (int k = 0; k < kRowMaxVec; ++k) {
+  for (int k = 0; k < MAXVEC; ++k) {
     const int i = threadIdx.x + k * kRowThreads;
     if (i < nvec) m = fmaxf(m, fmaxf(fmaxf(fabsf(y[k].x), fabsf(y[k].y)), fmaxf(fabsf(y[k].z), fabsf(y[k].w))));
   }
@@ -51,7 +52,7 @@ ZI_DEV void store_row_e4m3(const float4* y, int nvec, float* red, uint8_t* q, fl
   const float inv = zero ? 0.f : __fdiv_rn(448.f, amax);
   if (threadIdx.x == 0) *scale = zero ? 1.f : __fdiv_rn(amax, 448.f);
 #pragma unroll
-  for (int k = 0; k < kRowMaxVec; ++k) {
+  for (int k = 0; k < MAXVEC; ++k) {
     const int i = threadIdx.x + k * kRowThreads;
     if (i < nvec) {
       const float4 v = y[k];
@@ -121,17 +122,18 @@ __global__ void __launch_bounds__(kRowThreads) rms_mod_kernel(const TIn* __restr
 }
 
 // Per-row e4m3 quantisation of x [rows][D] (fp32 or bf16): q [rows][D] codes and
-// s [rows] scales, as store_row_e4m3 forms them.  One CTA per row.
-template <typename TIn>
+// s [rows] scales, as store_row_e4m3 forms them.  One CTA per row; rows up to
+// kRowThreads * MAXVEC * 4 wide.
+template <typename TIn, int MAXVEC>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_e4m3_kernel(const TIn* __restrict__ x, int D,
                                                                          uint8_t* __restrict__ q,
                                                                          float* __restrict__ s) {
   __shared__ float red[kRowThreads / 32];
   const int row = blockIdx.x;
   const int nvec = D >> 2;
-  float4 v[kRowMaxVec];
+  float4 v[MAXVEC];
 #pragma unroll
-  for (int k = 0; k < kRowMaxVec; ++k) {
+  for (int k = 0; k < MAXVEC; ++k) {
     const int i = threadIdx.x + k * kRowThreads;
     v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i < nvec) {
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_e4m3_kernel(const T
       }
     }
   }
-  store_row_e4m3(v, nvec, red, q + size_t(row) * D, s + row);
+  store_row_e4m3<MAXVEC>(v, nvec, red, q + size_t(row) * D, s + row);
 }
 
 enum NextNorm : int { NEXT_NONE = 0, NEXT_RMS = 1, NEXT_LAYERNORM = 2 };

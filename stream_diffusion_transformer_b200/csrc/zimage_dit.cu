@@ -276,6 +276,19 @@ int run_rms_mod(const TIn* x, int rows, int D, const uint16_t* gain, const float
   return launched(ZI_KERNEL_PRE_NORM, st);
 }
 
+// Per-row e4m3 codes and scales of a [rows, cols] fp32 or bf16 matrix (cols <= 16384).
+constexpr int kQuantMaxCols = kRowThreads * 16 * 4;
+template <typename TIn>
+int run_quantize(const TIn* x, int rows, int cols, uint8_t* q, float* sc, cudaStream_t st) {
+  if (rows <= 0) return ZI_OK;
+  prof_pre(st);
+  if (cols <= kRowThreads * kRowMaxVec * 4)
+    quantize_rows_e4m3_kernel<TIn, kRowMaxVec><<<rows, kRowThreads, 0, st>>>(x, cols, q, sc);
+  else
+    quantize_rows_e4m3_kernel<TIn, 16><<<rows, kRowThreads, 0, st>>>(x, cols, q, sc);
+  return launched(ZI_KERNEL_QUANTIZE, st);
+}
+
 int run_post(const PostParams& p, int rows, cudaStream_t st) {
   if (rows <= 0) return ZI_OK;
   prof_pre(st);
@@ -289,7 +302,8 @@ constexpr size_t kAlign = 1024;
 inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Ws {
-  size_t mod, c, silu, hid, lens, pos, rope, x, h, hs, qkv, att, o, u, tok, capn, split_cnt, split_part, total;
+  size_t mod, c, silu, hid, lens, pos, rope, x, h, hs, qkv, att, o, u, q8, q8s, tok, capn, split_cnt, split_part,
+      total;
 };
 
 Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int mod_cols) {
@@ -316,6 +330,9 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.att = o; o = up(o + rows * D * 2);
   w.o = o; o = up(o + rows * D * 2);
   w.u = o; o = up(o + rows * Fp * 2);
+  // e4m3 codes of the attention output or of u (never live together) and their row scales
+  w.q8 = o; o = up(o + rows * (Fp > D ? Fp : D));
+  w.q8s = o; o = up(o + rows * 4);
   w.tok = o; o = up(o + (model ? size_t(batch) * s_img * size_t(4 * cfg.in_ch) * 2 : 0));
   w.capn = o; o = up(o + (model ? size_t(batch) * s_txt * size_t(cfg.cap_dim) * 2 : 0));
   w.split_cnt = o; o = up(o + size_t(kSplitSlots) * 4);
@@ -349,9 +366,12 @@ bool block_ptrs_ok(const zi_block_weights* w, bool need_mod) {
     if (!p) return false;
   if (need_mod && (!w->w_ada || !w->b_ada)) return false;
   if ((w->w_ada == nullptr) != (w->b_ada == nullptr)) return false;
-  // e4m3 projections: all four of w_qkv8, s_qkv, w13_8, s_13, or none
+  // e4m3 projections: all four of w_qkv8, s_qkv, w13_8, s_13, or none; then optionally
+  // all four of w_out8, s_out, w2_8, s_2
   const int nf8 = (w->w_qkv8 != nullptr) + (w->s_qkv != nullptr) + (w->w13_8 != nullptr) + (w->s_13 != nullptr);
   if (nf8 != 0 && nf8 != 4) return false;
+  const int nf8b = (w->w_out8 != nullptr) + (w->s_out != nullptr) + (w->w2_8 != nullptr) + (w->s_2 != nullptr);
+  if (nf8b != 0 && (nf8b != 4 || nf8 != 4)) return false;
   return true;
 }
 
@@ -361,6 +381,8 @@ bool block_align_ok(const zi_block_weights* w) {
     if (!aligned16(p)) return false;
   if (w->w_ada && !aligned16(w->w_ada)) return false;
   if (w->w_qkv8 && (!aligned16(w->w_qkv8) || !aligned16(w->s_qkv) || !aligned16(w->w13_8) || !aligned16(w->s_13)))
+    return false;
+  if (w->w_out8 && (!aligned16(w->w_out8) || !aligned16(w->s_out) || !aligned16(w->w2_8) || !aligned16(w->s_2)))
     return false;
   return true;
 }
@@ -374,8 +396,10 @@ struct NextNormSpec {
   bool f8 = false;     // the next block takes e4m3 h (NEXT_RMS only)
 };
 
-// A block runs its QKV and FFN w1|w3 projections in e4m3 when it carries e4m3 weights.
+// A block runs its QKV and FFN w1|w3 projections in e4m3 when it carries e4m3 weights
+// for them, and also its output projection and FFN w2 when it carries those too.
 inline bool block_f8(const zi_block_weights* w) { return w && w->w_qkv8 != nullptr; }
+inline bool block_f8_all(const zi_block_weights* w) { return block_f8(w) && w->w_out8 != nullptr; }
 
 // One block over `rows` rows of the token buffer starting at global row `row_off`.
 // Pointers are local (row 0 = global row row_off).  h must already hold the
@@ -391,6 +415,8 @@ struct BlockCtx {
   uint16_t *h, *qkv, *att, *o, *u;
   uint8_t* hq;  // the same buffer as h, as e4m3 codes (D bytes per row) for e4m3 blocks
   float* hs;    // per-row scales of hq
+  uint8_t* q8;  // e4m3 codes of att or u (all-e4m3 blocks), and ...
+  float* q8s;   // ... their per-row scales
   const float2* rope;  // pair-major [head_dim / 2][rope_n]
   int rope_n;
   const float* mod;  // this block's 4D modulation inside the per-batch vector, or null
@@ -427,8 +453,18 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
   }
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len,
                        b.kv_len, st, b.split));
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D,
-                                  epi_plain(b.o, D), st, b.split)));
+  const bool f8all = block_f8_all(b.w);
+  if (f8all) {
+    ZI_TRY(run_quantize(b.att, b.rows, D, b.q8, b.q8s, st));
+    EpiParams eo = epi_plain(b.o, D);
+    eo.a_scale = b.q8s;
+    eo.b_scale = b.w->s_out;
+    ZI_TRY((run_gemm<256, EPI_BF16, true>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.q8, b.w->w_out8, b.rows, D, D,
+                                          eo, st, b.split)));
+  } else {
+    ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_OUT, b.att, b.w->w_out, b.rows, D, D,
+                                    epi_plain(b.o, D), st, b.split)));
+  }
   PostParams pa;
   memset(&pa, 0, sizeof(pa));
   pa.x_in = b.x_in;
@@ -461,8 +497,17 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
     ZI_TRY((run_gemm<256, EPI_SWIGLU>(b.dev, BIT_GEMM_SWIGLU, ZI_KERNEL_GEMM_FFN_UP, b.h, b.w->w13, b.rows, 2 * Fp,
                                       D, epi_plain(b.u, Fp), st, b.split)));
   }
-  ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp,
-                                  epi_plain(b.o, D), st, b.split)));
+  if (f8all) {
+    ZI_TRY(run_quantize(b.u, b.rows, Fp, b.q8, b.q8s, st));
+    EpiParams ed = epi_plain(b.o, D);
+    ed.a_scale = b.q8s;
+    ed.b_scale = b.w->s_2;
+    ZI_TRY((run_gemm<256, EPI_BF16, true>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.q8, b.w->w2_8, b.rows, D,
+                                          Fp, ed, st, b.split)));
+  } else {
+    ZI_TRY((run_gemm<256, EPI_BF16>(b.dev, BIT_GEMM_BF16, ZI_KERNEL_GEMM_FFN_DOWN, b.u, b.w->w2, b.rows, D, Fp,
+                                    epi_plain(b.o, D), st, b.split)));
+  }
   PostParams pf = pa;
   pf.x_in = b.x_out;
   pf.g_post = b.w->g_ffn2;
@@ -668,18 +713,13 @@ int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m,
 int zi_quantize_rows_e4m3(const void* d_x, int x_bf16, int rows, int cols, uint8_t* d_q, float* d_s,
                           zi_stream_t stream) {
   if (!d_x || !d_q || !d_s || rows < 0 || cols <= 0 || (x_bf16 != 0 && x_bf16 != 1)) return ZI_ERR_ARG;
-  if (cols % 4 || cols > kRowThreads * kRowMaxVec * 4) return ZI_ERR_SHAPE;
+  if (cols % 4 || cols > kQuantMaxCols) return ZI_ERR_SHAPE;
   if (!aligned16(d_x) || !aligned16(d_q) || !aligned16(d_s)) return ZI_ERR_ALIGN;
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
-  if (rows == 0) return ZI_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  prof_pre(st);
-  if (x_bf16)
-    quantize_rows_e4m3_kernel<uint16_t><<<rows, kRowThreads, 0, st>>>(static_cast<const uint16_t*>(d_x), cols, d_q, d_s);
-  else
-    quantize_rows_e4m3_kernel<float><<<rows, kRowThreads, 0, st>>>(static_cast<const float*>(d_x), cols, d_q, d_s);
-  return launched(ZI_KERNEL_QUANTIZE, st);
+  if (x_bf16) return run_quantize(static_cast<const uint16_t*>(d_x), rows, cols, d_q, d_s, st);
+  return run_quantize(static_cast<const float*>(d_x), rows, cols, d_q, d_s, st);
 }
 
 int zi_gemm_e4m3(const uint8_t* d_a, const float* d_sa, const uint8_t* d_b, const float* d_sb, uint16_t* d_c, int m,
@@ -768,6 +808,8 @@ int zi_block_forward(const zi_config* cfg, const zi_block_weights* w, const floa
   b.h = reinterpret_cast<uint16_t*>(ws + L.h);
   b.hq = ws + L.h;
   b.hs = reinterpret_cast<float*>(ws + L.hs);
+  b.q8 = ws + L.q8;
+  b.q8s = reinterpret_cast<float*>(ws + L.q8s);
   b.qkv = reinterpret_cast<uint16_t*>(ws + L.qkv);
   b.att = reinterpret_cast<uint16_t*>(ws + L.att);
   b.o = reinterpret_cast<uint16_t*>(ws + L.o);
@@ -840,6 +882,13 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     if (block_f8(&w->ctx[i]) != f8) return ZI_ERR_ARG;
   for (int i = 0; i < cfg->n_main; ++i)
     if (block_f8(&w->main[i]) != f8) return ZI_ERR_ARG;
+  const bool f8all = block_f8_all(&w->main[0]);
+  for (int i = 0; i < cfg->n_noise; ++i)
+    if (block_f8_all(&w->noise[i]) != f8all) return ZI_ERR_ARG;
+  for (int i = 0; i < cfg->n_ctx; ++i)
+    if (block_f8_all(&w->ctx[i]) != f8all) return ZI_ERR_ARG;
+  for (int i = 0; i < cfg->n_main; ++i)
+    if (block_f8_all(&w->main[i]) != f8all) return ZI_ERR_ARG;
   if (!aligned16(w->x_emb_w) || !aligned16(w->cap_w) || !aligned16(w->final_w) || !aligned16(w->final_ada_w) ||
       !aligned16(w->x_emb_b) || !aligned16(w->cap_b) || !aligned16(w->cap_norm) || !aligned16(d_txt) ||
       !aligned16(d_latent) || !aligned16(d_out))
@@ -982,6 +1031,7 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
   base.kv_len = lens;
   base.split = split;
 
+  const int Fp_ = zi_ffn_padded(cfg->ffn);
   auto segment_ctx = [&](int row_off, int nrows, int seglen) {
     BlockCtx b = base;
     b.rows = nrows;
@@ -991,6 +1041,8 @@ int model_forward_impl(const zi_config* cfg, const zi_model_weights* w, int batc
     b.h = h + size_t(row_off) * D;
     b.hq = ws + L.h + size_t(row_off) * D;  // e4m3 rows are D bytes
     b.hs = hs + row_off;
+    b.q8 = ws + L.q8 + size_t(row_off) * (Fp_ > D ? Fp_ : D);
+    b.q8s = reinterpret_cast<float*>(ws + L.q8s) + row_off;
     b.qkv = qkv + size_t(row_off) * 3 * D;
     b.att = att + size_t(row_off) * D;
     b.o = o + size_t(row_off) * D;

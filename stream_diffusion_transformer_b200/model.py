@@ -71,10 +71,11 @@ class DeviceBlock:
 
     fp8=True also stores e4m3 codes of the fused qkv and w13 with one scale per
     output channel (zi_quantize_rows_e4m3); the block then runs those two
-    projections in e4m3."""
+    projections in e4m3.  fp8="all" does the same for w_out and w2, so every
+    projection of the block runs in e4m3."""
 
     def __init__(self, cfg: abi.ZiConfig, prefix: str, bits: Dict[str, Bits], modulated: bool, device,
-                 fp8: bool = False):
+                 fp8=False):
         D, F = cfg.dim, cfg.ffn
         Fp = abi.ffn_padded(F)
         a = f"{prefix}.attention"
@@ -102,7 +103,10 @@ class DeviceBlock:
             self.t["b_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.bias"], device)
         self.modulated = modulated
         if fp8:
-            for src, q, sc in (("w_qkv", "w_qkv8", "s_qkv"), ("w13", "w13_8", "s_13")):
+            groups = [("w_qkv", "w_qkv8", "s_qkv"), ("w13", "w13_8", "s_13")]
+            if fp8 == "all":
+                groups += [("w_out", "w_out8", "s_out"), ("w2", "w2_8", "s_2")]
+            for src, q, sc in groups:
                 self.t[q], self.t[sc] = quantize_rows_e4m3(self.t[src])
         self.fp8 = fp8
         self.struct = abi.ZiBlockWeights(**{f: (self.t[f].data_ptr() if f in self.t else None)
@@ -116,10 +120,11 @@ class DiT:
     """The S3-DiT transformer on one GPU, weights resident in HBM."""
 
     def __init__(self, cfg: abi.ZiConfig, fetch: Callable[[Sequence[str]], Dict[str, Bits]], device="cuda",
-                 fp8: bool = False):
+                 fp8=False):
         """fetch(keys) -> {key: bf16 bits} is called once per block and once for the rest,
         so a 12 GB model never has to sit in host memory at once.  fp8=True runs every
-        block's QKV and FFN w1|w3 projections in e4m3 (see DeviceBlock)."""
+        block's QKV and FFN w1|w3 projections in e4m3, fp8="all" every block
+        projection (see DeviceBlock)."""
         self.cfg = cfg
         self.device = torch.device(device)
         abi.lib()
