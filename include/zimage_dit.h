@@ -248,7 +248,8 @@ ZI_API int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* 
 /* FlowMatch-Euler step in place (z-image-turbo-mnn "Scheduler"):
  *   y = d_out_uncond ? d_out_uncond + guidance (d_out_cond - d_out_uncond) : d_out_cond
  *   d_x += (sigma_next - sigma) * (-y)          (n fp32 elements)
- * d_out_uncond may be NULL (no CFG; guidance ignored). */
+ * d_out_uncond may be NULL (no CFG; guidance ignored).  n == 0 enqueues nothing and
+ * returns ZI_OK whatever the pointers. */
 ZI_API int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond, float guidance, double sigma,
                   double sigma_next, size_t n, zi_stream_t stream);
 

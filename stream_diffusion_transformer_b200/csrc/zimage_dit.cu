@@ -1157,10 +1157,10 @@ int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* w, int 
 
 int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond, float guidance, double sigma,
                   double sigma_next, size_t n, zi_stream_t stream) {
+  if (n == 0) return ZI_OK;  // nothing to do; the pointers of empty arrays may be NULL
   if (!d_x || !d_out_cond) return ZI_ERR_ARG;
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
-  if (n == 0) return ZI_OK;
   const float dt = float(sigma_next - sigma);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   prof_pre(st);

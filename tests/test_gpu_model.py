@@ -174,3 +174,39 @@ def test_graph_captured_loop_matches_eager():
         torch.cuda.synchronize()
         assert torch.isfinite(got).all()
         assert torch.equal(got, eager)
+
+
+@pytest.mark.parametrize("t", [0.0, 1.0])
+def test_degenerate_one_image_token_one_text_token(t):
+    """The smallest sequence: a 2x2 latent (one image token) and one text token, at the
+    timestep's end points t = 0 and t = 1; batch 2 with identical elements gives
+    identical outputs."""
+    from stream_diffusion_transformer_b200 import model
+    d = zi.TINY_R
+    bits = zi.make_weights(d, seed=12)
+    dit = model.DiT(model.make_config(d), lambda keys: {k: bits[k] for k in keys})
+    lat = np.repeat(zi.make_latent(d, 1, 2, 2, seed=12), 2, axis=0)
+    txt = np.repeat(zi.make_text(d, 1, 1, seed=12), 2, axis=0)
+    tt = np.array([t, t], dtype=np.float32)
+    out = dit.forward(torch.from_numpy(np.ascontiguousarray(lat)).cuda(), torch.from_numpy(tt).cuda(),
+                      torch.from_numpy(np.ascontiguousarray(txt).view(np.int16)).cuda().view(torch.bfloat16))
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    np.testing.assert_array_equal(got[0], got[1])
+    want = ref.model_forward(lat[:1].astype(np.float64), tt[:1].astype(np.float64),
+                             zi.bf16_bits_to_f32(txt[:1]).astype(np.float64), ref.Weights(bits), d)
+    assert_parity(got[:1].astype(np.float64), want, rel=3e-2, cos=0.995, what=f"1 + 1 tokens, t={t}")
+
+
+def test_empty_calls_enqueue_nothing():
+    """Zero-sized work is accepted and launches nothing (no kernel, no error)."""
+    from stream_diffusion_transformer_b200 import abi, model
+    a = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")  # real buffers; M = 0 rows are used
+    b = torch.zeros((256, 64), dtype=torch.bfloat16, device="cuda")
+    c = torch.zeros((1, 256), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros(16, device="cuda")
+    with abi.Profile(capacity=8) as prof:
+        abi.call("zi_gemm_bf16", model._p(a), model._p(b), model._p(c), 0, 256, 64, model._stream())
+        model.euler_step(x[:0], x[:0], None, 0.0, 1.0, 0.5)
+    torch.cuda.synchronize()
+    assert prof.kinds == []
