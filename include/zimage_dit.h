@@ -362,7 +362,8 @@ enum zi_kernel_kind {
   ZI_KERNEL_GEMM = 16,          /* zi_gemm_bf16 */
   ZI_KERNEL_TEXT_PAD = 17,      /* cap_pad_token into padded text rows */
   ZI_KERNEL_SPLIT_CLEAR = 18,   /* zero the GEMM split-tail counters (once per forward) */
-  ZI_KERNEL_QUANTIZE = 19       /* zi_quantize_rows_e4m3 */
+  ZI_KERNEL_QUANTIZE = 19,      /* zi_quantize_rows_e4m3 */
+  ZI_KERNEL_SELFTEST = 20       /* zi_watchdog_selftest */
 };
 
 /* Start recording launch timings on this host thread: from the next kernel the
@@ -379,6 +380,15 @@ ZI_API int zi_profile_begin(int capacity);
 ZI_API int zi_profile_end(float* h_ms, int* h_kinds, int capacity, int* h_count);
 
 /* ---------------------------------------------------------------- device status */
+
+/* Failure-detection self-test: enqueues one kernel whose single waiting thread
+ * spins on an mbarrier that nothing completes, with the library's bounded wait
+ * (here limit_us microseconds, 1 .. 2,000,000; else ZI_ERR_ARG).  When the
+ * limit runs out the kernel records a timeout in the device error word (raw
+ * code 6) and returns, so the context stays usable: zi_device_status() then
+ * reports ZI_ERR_TIMEOUT, and until zi_clear_device_status() every pipeline
+ * kernel of the library exits at once without touching memory. */
+ZI_API int zi_watchdog_selftest(int limit_us, zi_stream_t stream);
 
 /* Reads (synchronously) the device error word of the current device: ZI_OK, or
  * ZI_ERR_TIMEOUT if a kernel's bounded pipeline wait ran out since the last

@@ -83,6 +83,7 @@ _SIGS = {
     "zi_attention_varlen": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_profile_begin": (c_int, [c_int]),
     "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),
+    "zi_watchdog_selftest": (c_int, [c_int, c_void_p]),
     "zi_device_status": (c_int, [POINTER(c_int)]),
     "zi_clear_device_status": (c_int, []),
 }
@@ -164,7 +165,7 @@ KERNEL_NAMES = {
     1: "gemm_qkv_qknorm_rope", 2: "attention", 3: "gemm_out_proj", 4: "gemm_ffn_up_swiglu",
     5: "gemm_ffn_down", 6: "post_norm_residual", 7: "pre_norm", 8: "adaln_gemv", 9: "timestep_mlp",
     10: "rope_table", 11: "positions", 12: "patchify", 13: "gemm_embed", 14: "gemm_final_unpatchify",
-    15: "euler", 16: "gemm", 17: "text_pad", 18: "split_clear", 19: "quantize_e4m3",
+    15: "euler", 16: "gemm", 17: "text_pad", 18: "split_clear", 19: "quantize_e4m3", 20: "watchdog_selftest",
 }
 
 

@@ -28,6 +28,7 @@ enum : unsigned int {
   ZI_DEVERR_TIMEOUT_EPILOGUE = 3,
   ZI_DEVERR_TIMEOUT_SOFTMAX = 4,
   ZI_DEVERR_TIMEOUT_DRAIN = 5,
+  ZI_DEVERR_TIMEOUT_SELFTEST = 6,  // zi_watchdog_selftest: a wait that nothing completes
 };
 
 // A wait gives up after this many nanoseconds of %globaltimer.
@@ -81,7 +82,8 @@ ZI_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of the given parity to complete.  Returns false (after
 // recording `code` and raising *abort) if the limit runs out or another thread
 // of the CTA already aborted.
-ZI_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned int code) {
+ZI_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned int code,
+                      unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
@@ -89,7 +91,7 @@ ZI_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsig
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         raise_device_error(code);
         *abort = 1;
         return false;

@@ -303,6 +303,20 @@ __global__ void positions_varlen_kernel(int s_txt, int grid_h, int grid_w, const
   pos[3 * t + 2] = a2;
 }
 
+// Failure-detection self-test: one thread waits on an mbarrier that nothing
+// arrives on; the bounded wait gives up after limit_ns, records
+// ZI_DEVERR_TIMEOUT_SELFTEST in the device error word and the kernel returns.
+__global__ void watchdog_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag, ZI_DEVERR_TIMEOUT_SELFTEST, limit_ns);
+  }
+}
+
 __global__ void zero_ints_kernel(int* __restrict__ p, int n) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0;
 }

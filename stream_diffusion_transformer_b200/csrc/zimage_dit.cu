@@ -1214,6 +1214,16 @@ int zi_profile_end(float* h_ms, int* h_kinds, int capacity, int* h_count) {
   return st;
 }
 
+int zi_watchdog_selftest(int limit_us, zi_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000) return ZI_ERR_ARG;
+  DevInfo* dev;
+  ZI_TRY(current_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  prof_pre(st);
+  watchdog_selftest_kernel<<<1, 32, 0, st>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
+  return launched(ZI_KERNEL_SELFTEST, st);
+}
+
 int zi_device_status(int* h_code) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, zi::g_zi_error, sizeof(v)) != cudaSuccess) return ZI_ERR_CUDA;

@@ -111,6 +111,8 @@ def test_argument_checks_need_no_gpu(abi):
     assert L.zi_euler_step(None, None, None, 0.0, 1.0, 0.5, 4, None) == abi.ZI_ERR_ARG
     assert L.zi_block_forward(ctypes.byref(c), None, None, None, 1, 16, None, None, None, 0, None) == abi.ZI_ERR_ARG
     assert L.zi_sigmas(0, 3.0, None) == abi.ZI_ERR_ARG
+    assert L.zi_watchdog_selftest(0, None) == abi.ZI_ERR_ARG
+    assert L.zi_watchdog_selftest(3000000, None) == abi.ZI_ERR_ARG
 
 
 def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
