@@ -227,6 +227,37 @@ class DiT:
         return out
 
 
+def denoise_cfg_split(latent: torch.Tensor, n_steps: int, shift: float, guidance: float,
+                      forward: Callable[[torch.Tensor, torch.Tensor], torch.Tensor],
+                      euler: Optional[Callable] = None, group=None) -> torch.Tensor:
+    """Classifier-free guidance with the two branches on two ranks (one GPU each):
+    rank 0 runs the conditional forward, rank 1 the unconditional one, each on its
+    own full replica of the weights; after every forward the two raw outputs are
+    exchanged with one all-gather (torch.distributed over NCCL on GPUs; 4 MB per
+    step at 2048x2048) and both ranks apply the same guided Euler step, so their
+    latents stay identical.
+
+    forward(x, t) -> raw output of x's shape, for this rank's branch (for example
+    lambda x, t: dit.forward(x, t, txt_of_this_branch)).  euler(x, y_cond, y_uncond,
+    guidance, sigma, sigma_next) updates x in place; by default zi_euler_step.
+    Returns the final latent (a new tensor)."""
+    import torch.distributed as dist
+    if dist.get_world_size(group) != 2:
+        raise ValueError("the CFG split runs on exactly two ranks")
+    if euler is None:
+        euler = lambda x, yc, yu, g, s0, s1: euler_step(x, yc, yu, g, s0, s1)
+    sig = abi.sigmas(n_steps, shift)
+    x = latent.clone()
+    t = torch.empty(x.shape[0], dtype=torch.float32, device=x.device)
+    both = [torch.empty_like(x), torch.empty_like(x)]
+    for i in range(n_steps):
+        t.fill_(1.0 - sig[i])
+        y = forward(x, t)
+        dist.all_gather(both, y.contiguous(), group=group)  # [conditional, unconditional]
+        euler(x, both[0], both[1], float(guidance), sig[i], sig[i + 1])
+    return x
+
+
 class DenoiseGraph:
     """DiT.denoise captured once as a CUDA graph and replayed: all n_steps forwards,
     their Euler steps (sigmas baked in) and, with guidance, the CFG combines, for
