@@ -194,7 +194,10 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const void* A, const void* B,
   return launched(kind, st);
 }
 
-static_assert(size_t(attn::kSlotF4) * 16 >= size_t(128) * 256 * 4, "a split slot holds a GEMM tile partial");
+// bytes of one split-tail slot: a GEMM tile partial (128 x 256 fp32) or an attention
+// piece (O of two query tiles plus their row max and sum), whichever is larger
+constexpr size_t kSplitSlotBytes = size_t(128) * 256 * 4 > size_t(attn::kSlotF4) * 16 ? size_t(128) * 256 * 4
+                                                                                       : size_t(attn::kSlotF4) * 16;
 
 // Zeroes the split-tail counters of a workspace (once per forward; every tile's
 // finisher puts its counter back to zero).
@@ -336,9 +339,7 @@ Ws carve(const zi_config& cfg, int batch, int s_img, int s_txt, bool model, int 
   w.tok = o; o = up(o + (model ? size_t(batch) * s_img * size_t(4 * cfg.in_ch) * 2 : 0));
   w.capn = o; o = up(o + (model ? size_t(batch) * s_txt * size_t(cfg.cap_dim) * 2 : 0));
   w.split_cnt = o; o = up(o + size_t(kSplitSlots) * 4);
-  // partial slots of the split tails: a GEMM tile (128 x 256 fp32) or an attention
-  // piece (O of two query tiles plus their row max and sum), whichever is larger
-  w.split_part = o; o = up(o + size_t(kSplitSlots) * size_t(attn::kSlotF4) * 16);
+  w.split_part = o; o = up(o + size_t(kSplitSlots) * kSplitSlotBytes);
   w.total = o;
   return w;
 }
