@@ -24,6 +24,7 @@ import argparse
 import dataclasses
 import datetime
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -75,12 +76,17 @@ def load_peaks():
 
 
 def kernel_source_hash(files) -> str:
-    """Hash of the CUDA sources a kernel is built from (names under the package's csrc/)."""
+    """Hash of the CUDA sources a kernel is built from (names under the package's csrc/),
+    over the code only: comments and whitespace are dropped, so editing a comment does
+    not mark recorded counters as stale, while any change to the code does."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "stream_diffusion_transformer_b200", "csrc")
     for name in sorted(files):
-        with open(os.path.join(cdir, name), "rb") as fh:
-            h.update(name.encode() + fh.read())
+        with open(os.path.join(cdir, name)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)   # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                  # line comments
+        h.update(name.encode() + " ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -4,13 +4,13 @@
 // in three warpgroups; registers move from the third to the first two with
 // setmaxnreg (launch 168 per thread; softmax 216, TMA/MMA 56):
 //   warp 8      TMA: both Q tiles once, then K tiles (128 keys each) into a
-//               2-deep ring, straight out of the fused [rows, 3D] projection
+//               3-deep ring, straight out of the fused [rows, 3D] projection
 //               buffer (the head's 128 columns as two 64-wide swizzled boxes)
 //   warp 9      TMEM allocator + tcgen05.mma issuer.  TMEM: S_A, S_B, O_A, O_B,
 //               128 columns each.  Per key tile j the tensor core runs
 //                 S_A(j+1) = Q_A K^T, O_B += P_B(j) V, S_B(j+1) = Q_B K^T, O_A += P_A(j+1) V
 //               so each tile's softmax has the other tile's two MMAs to hide behind.
-//   warp 10     TMA for the V ring (warp 8 then only loads Q and K)
+//   warp 10     TMA for the 2-deep V ring (warp 8 then only loads Q and K)
 //   warp 11     idle
 //   warps 0..3  softmax of tile A, warps 4..7 softmax of tile B: one thread per
 //               query row (its TMEM lane); online softmax in the exp2 domain with a

@@ -1,15 +1,18 @@
-// Persistent bf16 GEMM for sm_100a with fused epilogues:  C[M, N] = A[M, K] * B[N, K]^T.
+// Persistent GEMM for sm_100a with fused epilogues:  C[M, N] = A[M, K] * B[N, K]^T,
+// operands bf16 (kind::f16) or e4m3 with per-row scales (kind::f8f6f4).
 //
 // A is the activation (row-major, K contiguous); B is a weight in the
 // checkpoint's own [out, in] orientation, which is exactly the K-major operand
 // tcgen05 wants, so weights are used as stored.
 //
-// One CTA per SM, 6 warps:
-//   warp 0      TMA producer: 128 x 64 A tile + BN x 64 B tile per stage,
-//               128-byte swizzle, STAGES-deep mbarrier ring
+// One CTA per SM, 10 warps:
+//   warp 0      TMA producer: a 128-row A tile + a BN-row B tile of 128 bytes of K
+//               per stage (64 bf16 or 128 e4m3), 128-byte swizzle, STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//               (M = 128, N = BN, K = 16 per instruction; fp32 accumulator in TMEM)
-//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> fused math -> global
+//               (M = 128, N = BN, 32 bytes of K per instruction; fp32 accumulator in TMEM)
+//   warps 2..9  epilogue in two groups of four (each covers all 128 TMEM lanes and
+//               one half of the tile's columns): tcgen05.ld TMEM -> registers ->
+//               fused math -> global
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the epilogue
 // of tile i overlaps the main loop of tile i + 1.  Tiles are walked M-fastest
 // so that CTAs running at the same time share weight tiles through L2.
