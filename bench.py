@@ -423,12 +423,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                               "source": "Z-Image-Turbo repackaged for H3ddle, Measured performance"},
     }
     if world == 1 and not args.no_cpu_baseline:
+        # the oracle's block, repeated until at least 10 s of CPU work (at most 4 runs)
         step, sflops, sample = oracle_sample()
-        t0 = time.perf_counter()
-        step()
+        runs, t0 = 0, time.perf_counter()
+        while runs < 4 and (runs == 0 or time.perf_counter() - t0 < 10.0):
+            step()
+            runs += 1
         dt = time.perf_counter() - t0
-        line["cpu_baseline"] = {"value": sflops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-                                "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+        line["cpu_baseline"] = {"value": sflops * runs / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": f"{sample}, run {runs} times", "seconds": round(dt, 2)}
     print(json.dumps(line), flush=True)
 
 
