@@ -137,6 +137,42 @@ def block_forward(x: np.ndarray, W: ref.Weights, prefix: str, d, angles: np.ndar
     return x1 + gate_mlp * ref.rms_norm(f, W(f"{prefix}.ffn_norm2.weight"))
 
 
+def block_forward_rows(x: np.ndarray, W: ref.Weights, prefix: str, d, angles: np.ndarray,
+                       c: Optional[np.ndarray], rows: np.ndarray, all: bool = False) -> np.ndarray:
+    """block_forward(x, ...)[rows] for the selected query rows only (keys and values
+    from every row).  Every step but attention is per row, and so is the e4m3
+    quantisation (one scale per row), so the selected rows' results are those of
+    the whole-sequence block."""
+    S, D = x.shape
+    H, hd = d.heads, d.head_dim
+    if c is not None:
+        scale_msa, gate_msa, scale_mlp, gate_mlp = ref.adaln(c, W, prefix)
+    else:
+        scale_msa = scale_mlp = 0.0
+        gate_msa = gate_mlp = 1.0
+    a = f"{prefix}.attention"
+    h = ref.rms_norm(x, W(f"{prefix}.attention_norm1.weight")) * (1.0 + scale_msa)
+    hq, hs = quantize_rows(h)
+    hd8 = dequantize_rows(hq, hs)  # the quantised h of every row
+    deq = lambda w: dequantize_rows(*quantize_rows(w))
+    k = ref.apply_rope(ref.rms_norm((hd8 @ deq(W(f"{a}.to_k.weight")).T).reshape(S, H, hd),
+                                    W(f"{a}.norm_k.weight")), angles)
+    v = (hd8 @ deq(W(f"{a}.to_v.weight")).T).reshape(S, H, hd)
+    q = (hd8[rows] @ deq(W(f"{a}.to_q.weight")).T).reshape(len(rows), H, hd)
+    q = ref.apply_rope(ref.rms_norm(q, W(f"{a}.norm_q.weight")), angles[rows])
+    att = ref.attention(q, k, v).reshape(len(rows), D)
+    o = fp8_linear(att, W(f"{a}.to_out.weight")) if all else ref.linear(att, W(f"{a}.to_out.weight"))
+    x1 = x[rows] + gate_msa * ref.rms_norm(o, W(f"{prefix}.attention_norm2.weight"))
+    h2 = ref.rms_norm(x1, W(f"{prefix}.ffn_norm1.weight")) * (1.0 + scale_mlp)
+    ff = f"{prefix}.feed_forward"
+    w13 = np.concatenate([W(f"{ff}.w1.weight"), W(f"{ff}.w3.weight")], axis=0)
+    g13 = fp8_linear(h2, w13)
+    F = d.ffn
+    u = ref.silu(g13[:, :F]) * g13[:, F:]
+    f = fp8_linear(u, W(f"{ff}.w2.weight")) if all else ref.linear(u, W(f"{ff}.w2.weight"))
+    return x1 + gate_mlp * ref.rms_norm(f, W(f"{prefix}.ffn_norm2.weight"))
+
+
 def model_forward(latent: np.ndarray, t: np.ndarray, txt: np.ndarray, W: ref.Weights, d,
                   all: bool = False) -> np.ndarray:
     """zimage_ref.model_forward with every block's QKV and FFN w1|w3 projections in e4m3

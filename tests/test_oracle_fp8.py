@@ -109,3 +109,18 @@ def test_all_projection_block_moves_further_from_bf16():
     y8a = f8.block_forward(x, W, "layers.0", d, ang, c, all=True)
     e = lambda y: np.linalg.norm((y - x) - (y16 - x)) / np.linalg.norm(y16 - x)
     assert 0 < e(y8) < e(y8a) < 0.2
+
+
+@pytest.mark.parametrize("all_", [False, True])
+def test_block_forward_rows_equals_whole_block(all_):
+    """Selecting query rows gives exactly those rows of the whole-sequence e4m3 block
+    (quantisation is per row, attention takes keys and values from every row)."""
+    d = zi.TINY_R
+    W = ref.Weights(zi.make_weights(d, seed=6))
+    x = zi.make_stream(d, 1, 40, seed=6)[0].astype(np.float64)
+    c = zi.make_cond(d, 1, seed=6)[0].astype(np.float64)
+    ang = ref.rope_angles(ref.position_ids(8, 4, 8), d.rope_axes)
+    rows = np.array([0, 3, 17, 31, 39])
+    whole = f8.block_forward(x, W, "layers.0", d, ang, c, all=all_)
+    np.testing.assert_allclose(f8.block_forward_rows(x, W, "layers.0", d, ang, c, rows, all=all_), whole[rows],
+                               rtol=1e-12, atol=1e-12)
