@@ -188,6 +188,59 @@ def oracle_sample():
     return step, block_flops(S, d.dim, d.ffn), f"one main block (full width, {S} tokens, fp64 NumPy)"
 
 
+def run_oracle_workload(args):
+    """Times the CPU oracle (fp64 NumPy) on the small configurations, on this host's
+    cores: the tiny model's whole forward, one full-width main block at 1,152 tokens
+    (all BLAS threads and one), and one main block at 4,128 tokens, from which a full
+    4,128-token forward is extrapolated.  Prints one JSON line."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import zimage_ref as ref
+
+    def timed(fn, min_s=2.0):
+        fn()
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= min_s:
+                return dt / n
+
+    out = {"workload": "CPU oracle timings (fp64 NumPy)", "host_cpus": os.cpu_count(),
+           "affinity_cpus": len(os.sched_getaffinity(0)), "blas_threads": blas_threads()}
+    # the tiny model, whole forward (64 image + 32 text tokens)
+    d = zi.TINY
+    W = ref.Weights(zi.make_weights(d, seed=SEED))
+    lat = zi.make_latent(d, 1, 16, 16, seed=SEED).astype(np.float64)
+    txt = zi.bf16_bits_to_f32(zi.make_text(d, 1, 32, seed=SEED)).astype(np.float64)
+    tt = np.array([T_VALUE])
+    sec = timed(lambda: ref.model_forward(lat, tt, txt, W, d))
+    fl = forward_flops(d, 64, 32)
+    out["tiny_model_forward"] = {"ms": sec * 1e3, "gflops": fl / sec / 1e9, "flops": fl}
+    # one full-width main block at 1,024 + 128 and at 4,096 + 32 tokens
+    d = zi.FULL
+    W = ref.Weights(zi.make_weights(d, seed=SEED, keys=[k for k, _, _ in zi.block_specs("layers.0", d, True)],
+                                    threads=8))
+    for name, (gh, gw, st) in {"block_1152": (32, 32, 128), "block_4128": (64, 64, S_TXT)}.items():
+        S = gh * gw + st
+        x = zi.make_stream(d, 1, S, seed=SEED)[0].astype(np.float64)
+        c = zi.make_cond(d, 1, seed=SEED)[0].astype(np.float64)
+        ang = ref.rope_angles(ref.position_ids(st, gh, gw), d.rope_axes)
+        fl = block_flops(S, d.dim, d.ffn)
+        sec = timed(lambda: ref.block_forward(x, W, "layers.0", d, ang, c))
+        out[name] = {"tokens": S, "ms": sec * 1e3, "gflops": fl / sec / 1e9, "threads": blas_threads()}
+        if name == "block_1152":
+            with threadpool_limits(limits=1, user_api="blas"):
+                sec1 = timed(lambda: ref.block_forward(x, W, "layers.0", d, ang, c), min_s=1.0)
+            out[name + "_1thread"] = {"ms": sec1 * 1e3, "gflops": fl / sec1 / 1e9, "threads": 1,
+                                      "speedup_all_threads": sec1 / sec}
+    rate = out["block_4128"]["gflops"] * 1e9
+    full = forward_flops(d, (LAT_H // 2) * (LAT_W // 2), S_TXT)
+    out["full_forward_4128_extrapolated_s"] = full / rate
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
@@ -622,11 +675,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8", "fp8all"], default="forward",
+    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8", "fp8all", "oracle"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
                          "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens; "
-                         "cfg: one guidance step at 2048x2048, batch 2 x 16,896 tokens")
+                         "cfg: one guidance step at 2048x2048, batch 2 x 16,896 tokens; fp8 / fp8all: the "
+                         "forward with e4m3 projections; oracle: CPU oracle timings on this host")
     args = ap.parse_args()
+    if args.workload == "oracle":
+        run_oracle_workload(args)
+        return
     if args.workload == "block":
         run_block_workload(args)
         return
