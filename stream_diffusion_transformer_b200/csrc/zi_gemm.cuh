@@ -14,8 +14,9 @@
 //               one half of the tile's columns): tcgen05.ld TMEM -> registers ->
 //               fused math -> global
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the epilogue
-// of tile i overlaps the main loop of tile i + 1.  Tiles are walked M-fastest
-// so that CTAs running at the same time share weight tiles through L2.
+// of tile i overlaps the main loop of tile i + 1.  Tiles are walked along the
+// shorter output dimension first (tile_origin), so that CTAs running at the same
+// time share the larger operand's tiles through L2.
 #pragma once
 #include "zi_common.cuh"
 
@@ -265,10 +266,29 @@ struct TailSched {
   int tail_s;      // K pieces per tail tile (1 = no tail)
   int tail_items;  // CTAs [0, tail_items) each run piece c % s of tile dp_tiles + c / s
   int kb;          // k-blocks per tile
+  int num_n;       // N tiles
+  int n_fast;      // tile index walks N fastest (else M fastest)
 };
 
-inline TailSched make_tail_sched(int tiles, int grid, int kb, bool can_split) {
-  TailSched s{grid, tiles, 1, 0, kb};
+// Tile t covers rows [m0, m0 + BM) and columns [n0, n0 + BN).  The index walks the
+// shorter dimension of the output fastest, so that the CTAs running at the same
+// time share the tiles of the larger operand through L2 while the smaller one stays
+// resident: M-fastest when N > M (the weight is the larger operand), N-fastest when
+// M > N (then the activation is, e.g. FFN down's 4,128 x 10,240 input, which would
+// otherwise be re-read from DRAM for every wave).
+template <int BM, int BN>
+ZI_DEV void tile_origin(const TailSched& s, int num_m, int tile, int& m0, int& n0) {
+  if (s.n_fast) {
+    m0 = (tile / s.num_n) * BM;
+    n0 = (tile % s.num_n) * BN;
+  } else {
+    m0 = (tile % num_m) * BM;
+    n0 = (tile / num_m) * BN;
+  }
+}
+
+inline TailSched make_tail_sched(int tiles, int grid, int kb, bool can_split, int num_n, bool n_fast) {
+  TailSched s{grid, tiles, 1, 0, kb, num_n, n_fast ? 1 : 0};
   const int rounds = tiles / grid, rest = tiles - rounds * grid;
   if (!can_split || rest == 0 || grid > kSplitSlots) return s;
   int f = grid / rest;
@@ -382,7 +402,8 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
       bool ok = true;
       WorkWalker walk(sched, blockIdx.x);
       while (ok && walk.next(wi)) {
-        const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
+        int m0, n0;
+        tile_origin<BM, BN>(sched, num_m, wi.tile, m0, n0);
         const uint32_t bytes = L::kStage;
         for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
           const uint32_t s = it % STAGES, r = it / STAGES;
@@ -474,7 +495,8 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
       ++local;
       if (!mbar_wait(&tfull[acc], u & 1u, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
-      const int m0 = (wi.tile % num_m) * BM, n0 = (wi.tile / num_m) * BN;
+      int m0, n0;
+      tile_origin<BM, BN>(sched, num_m, wi.tile, m0, n0);
       const int row = m0 + row_in_tile;
       const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
       bool finish = true;

@@ -186,7 +186,7 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const void* A, const void* B,
   auto kern = GemmKernel<BN, EPI, F8>::fn;
   ZI_TRY(ensure_smem(dev, bit + (F8 ? 8u : 0u), kern, int(L::kBytes)));
   const int tiles = ((M + 127) / 128) * (N / BN);
-  const TailSched sched = make_tail_sched(tiles, dev->sms, K / BK, sk.partials != nullptr);
+  const TailSched sched = make_tail_sched(tiles, dev->sms, K / BK, sk.partials != nullptr, N / BN, M > N);
   int grid = tiles < dev->sms ? tiles : dev->sms;
   if (sched.tail_items > grid) grid = sched.tail_items;  // fewer tiles than SMs, each cut along K
   prof_pre(st);
