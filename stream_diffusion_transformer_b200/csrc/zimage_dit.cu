@@ -194,8 +194,10 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const void* A, const void* B,
   return launched(kind, st);
 }
 
-// bytes of one split-tail slot: a GEMM tile partial (128 x 256 fp32)
-constexpr size_t kSplitSlotBytes = size_t(128) * 256 * 4;
+// bytes of one split-tail slot: a GEMM tile partial (128 x 256 fp32) or an attention
+// piece (O of two query tiles plus their row max and sum), whichever is larger
+constexpr size_t kSplitSlotBytes = size_t(128) * 256 * 4 > size_t(attn::kSlotF4) * 16 ? size_t(128) * 256 * 4
+                                                                                       : size_t(attn::kSlotF4) * 16;
 
 // Zeroes the split-tail counters of a workspace (once per forward; every tile's
 // finisher puts its counter back to zero).
@@ -216,12 +218,12 @@ EpiParams epi_plain(void* out, int ldo) {
 
 // ---------------------------------------------------------------- attention
 
+// sk.partials == nullptr: no split of the ragged last wave.
 int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out, int dim, int heads, int batch,
-                  int nseg, const int* row0, const int* len, const int* kv_len, cudaStream_t st) {
-  // Q tiles and value halves: 64 columns x 128 rows per box; key halves: 64 x 64
-  CUtensorMap tm_q, tm_k;
-  ZI_TRY(make_map(&tm_q, qkv, uint64_t(3 * dim), uint64_t(qkv_rows), uint64_t(3 * dim) * 2, 64, 128));
-  ZI_TRY(make_map(&tm_k, qkv, uint64_t(3 * dim), uint64_t(qkv_rows), uint64_t(3 * dim) * 2, 64, 64));
+                  int nseg, const int* row0, const int* len, const int* kv_len, cudaStream_t st,
+                  SplitScratch sk = SplitScratch{nullptr, nullptr}) {
+  CUtensorMap tm;
+  ZI_TRY(make_map(&tm, qkv, uint64_t(3 * dim), uint64_t(qkv_rows), uint64_t(3 * dim) * 2, 64, 128));
   ZI_TRY(ensure_smem(dev, BIT_ATTN, attention_kernel, int(attn::kSmemBytes)));
   AttnParams p;
   memset(&p, 0, sizeof(p));
@@ -238,12 +240,30 @@ int run_attention(DevInfo* dev, const uint16_t* qkv, int qkv_rows, uint16_t* out
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(128.0));
   p.q_tiles = qt;
   p.kv_len = kv_len;
+  p.pairs = (qt + 1) / 2;  // two query tiles per unit
   p.heads = heads;
-  // one CTA pair per (pair of query tiles, head, batch element)
-  const long long units = static_cast<long long>((qt + 1) / 2) * heads * batch;
-  if (units > 0x3fffffffLL) return ZI_ERR_SHAPE;
+  const long long units = static_cast<long long>(p.pairs) * heads * batch;
+  if (units > 0x7fffffffLL / attn::kMaxSplit) return ZI_ERR_SHAPE;
+  p.full_units = int(units);
+  p.split_s = 1;
+  const int G = dev->sms;
+  const int rest = int(units % G);
+  // fewest key tiles any element can have (each piece needs one)
+  const int min_kv = (nseg > 1 ? (len[0] + 127) / 128 : 0) + (kv_len ? 1 : (len[nseg - 1] + 127) / 128);
+  if (sk.partials && rest > 0 && G <= kSplitSlots) {
+    int f = G / rest;
+    if (f > attn::kMaxSplit) f = attn::kMaxSplit;
+    if (f > min_kv) f = min_kv;
+    if (f >= 2) {
+      p.full_units = int(units) - rest;
+      p.split_s = f;
+      p.part = sk.partials;
+      p.counters = sk.counters;
+    }
+  }
+  const int grid = p.full_units + (int(units) - p.full_units) * p.split_s;
   prof_pre(st);
-  attention_kernel<<<2 * int(units), attn::kThreads, attn::kSmemBytes, st>>>(tm_q, tm_k, p);
+  attention_kernel<<<grid, attn::kThreads, attn::kSmemBytes, st>>>(tm, p);
   return launched(ZI_KERNEL_ATTENTION, st);
 }
 
@@ -433,7 +453,7 @@ int run_block(const BlockCtx& b, const NextNormSpec& next, cudaStream_t st) {
                                    st, b.split)));
   }
   ZI_TRY(run_attention(b.dev, b.qkv, b.rows, b.att, D, b.cfg->heads, b.batch, b.nseg, b.seg_row0, b.seg_len,
-                       b.kv_len, st));
+                       b.kv_len, st, b.split));
   const bool f8all = block_f8_all(b.w);
   if (f8all) {
     ZI_TRY(run_quantize(b.att, b.rows, D, b.q8, b.q8s, st));
