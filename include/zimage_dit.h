@@ -258,6 +258,15 @@ ZI_API int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out
  * FastVideo handoff "Scheduler").  h_sigmas has n_steps + 1 entries. */
 ZI_API int zi_sigmas(int n_steps, double shift, double* h_sigmas);
 
+/* Host helper: the model timestep of each of the n_steps transformer calls of that
+ * schedule, t_i = 1 - sigma'_i (1 = clean), formed in double and rounded to float
+ * once: the card passes (1000 - 1000 sigma') / 1000 to the transformer
+ * (z-image-turbo-mnn "Scheduler"), and the zero-sigma end point gets no call
+ * (FastVideo handoff "Pinned official pipeline context").  h_t has n_steps
+ * entries, ready to copy into zi_model_forward's d_t.  ZI_ERR_ARG if n_steps <= 0,
+ * shift <= 0 or h_t is NULL. */
+ZI_API int zi_timesteps(int n_steps, double shift, float* h_t);
+
 /* ---------------------------------------------------------------- fixed-scratch variant
  * The pages describing the method have no counterpart to this entry point; it
  * exists for callers that cannot allocate device memory.  Examples: a plugin
@@ -305,9 +314,10 @@ ZI_API int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, floa
 
 /* C[M, N] = A[M, K] B[N, K]^T, bf16 in, fp32 accumulate, bf16 out (tcgen05).
  * K % 64 == 0, N % 256 == 0, M >= 1; rows are contiguous (strides K and N).
- * Same kernel and schedule as the projections of the forward: 128 x 256 tiles
- * on persistent CTAs, a ragged last wave cut along N into 128 x 128 or 128 x 64
- * sub-tiles. */
+ * Same kernel as the projections of the forward (128 x 256 tiles on persistent
+ * CTAs).  Inside the forward the ragged last wave of tiles is cut along K into
+ * pieces whose fp32 partials the last-arriving piece sums in piece order; this
+ * entry point has no workspace for those partials, so its tiles always run whole. */
 ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k,
                         zi_stream_t stream);
 

@@ -83,3 +83,44 @@ def position_ids_loop(s_txt: int, grid_h: int, grid_w: int) -> List[List[int]]:
     for j in range(s_txt):
         ids.append([j + 1, 0, 0])
     return ids
+
+
+def t_embed_loop(t: float, w1, b1, w2, b2, t_scale: float = 1000.0, max_period: float = 10000.0) -> List[float]:
+    """Conditioning vector of one timestep, written out element by element.
+
+    The model timestep t (1 = clean) is scaled by t_scale; entry k < half of the
+    sinusoid is cos(t_scale t f_k), entry half + k is sin(t_scale t f_k), with
+    f_k = max_period^(-k / half); then hidden unit j = SiLU(sum_k w1[j][k] e_k + b1[j])
+    and output i = sum_j w2[i][j] hidden_j + b2[i].  w1, w2 are [out][in] nested lists.
+    """
+    width = len(w1[0])
+    half = width // 2
+    e = [0.0] * width
+    for k in range(half):
+        arg = t * t_scale * math.exp(-math.log(max_period) * k / half)
+        e[k] = math.cos(arg)
+        e[half + k] = math.sin(arg)
+    hid = []
+    for j in range(len(w1)):
+        z = math.fsum(w1[j][k] * e[k] for k in range(width)) + b1[j]
+        hid.append(z / (1.0 + math.exp(-z)))
+    return [math.fsum(w2[i][j] * hid[j] for j in range(len(hid))) + b2[i] for i in range(len(w2))]
+
+
+def final_layer_loop(x_row: Sequence[float], c: Sequence[float], wa, ba, wf, bf, eps: float = 1e-6) -> List[float]:
+    """Final layer of one image token, element by element.
+
+    LayerNorm without affine (mean and biased variance over the row, eps inside the
+    root), scaled by (1 + s) with s_i = sum_k wa[i][k] SiLU(c_k) + ba[i], then the
+    linear map out_j = sum_i wf[j][i] y_i + bf[j].
+    """
+    n = len(x_row)
+    mu = math.fsum(x_row) / n
+    var = math.fsum((v - mu) ** 2 for v in x_row) / n
+    inv = 1.0 / math.sqrt(var + eps)
+    sc = [v / (1.0 + math.exp(-v)) for v in c]
+    y = []
+    for i in range(n):
+        s = math.fsum(wa[i][k] * sc[k] for k in range(len(sc))) + ba[i]
+        y.append((x_row[i] - mu) * inv * (1.0 + s))
+    return [math.fsum(wf[j][i] * y[i] for i in range(n)) + bf[j] for j in range(len(wf))]

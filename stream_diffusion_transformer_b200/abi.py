@@ -74,6 +74,7 @@ _SIGS = {
                                        c_void_p]),
     "zi_euler_step": (c_int, [c_void_p, c_void_p, c_void_p, c_float, c_double, c_double, c_size_t, c_void_p]),
     "zi_sigmas": (c_int, [c_int, c_double, POINTER(c_double)]),
+    "zi_timesteps": (c_int, [c_int, c_double, POINTER(c_float)]),
     "zi_positions": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
     "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
@@ -146,6 +147,14 @@ def model_workspace_size(cfg: ZiConfig, batch: int, lat_h: int, lat_w: int, s_tx
 def sigmas(n_steps: int, shift: float = 3.0):
     out = (c_double * (n_steps + 1))()
     call("zi_sigmas", n_steps, shift, out)
+    return list(out)
+
+
+def timesteps(n_steps: int, shift: float = 3.0):
+    """Model timestep of each transformer call of the schedule (zi_timesteps), as Python floats
+    holding the exact fp32 values."""
+    out = (c_float * n_steps)()
+    call("zi_timesteps", n_steps, shift, out)
     return list(out)
 
 

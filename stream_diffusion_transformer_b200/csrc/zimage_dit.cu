@@ -1179,6 +1179,14 @@ int zi_sigmas(int n_steps, double shift, double* h_sigmas) {
   return ZI_OK;
 }
 
+int zi_timesteps(int n_steps, double shift, float* h_t) {
+  if (n_steps <= 0 || !h_t || !(shift > 0.0)) return ZI_ERR_ARG;
+  std::vector<double> sig(size_t(n_steps) + 1);
+  ZI_TRY(zi_sigmas(n_steps, shift, sig.data()));
+  for (int i = 0; i < n_steps; ++i) h_t[i] = float(1.0 - sig[size_t(i)]);
+  return ZI_OK;
+}
+
 int zi_profile_begin(int capacity) {
   if (capacity <= 0) return ZI_ERR_ARG;
   if (g_prof.on) return ZI_ERR_ARG;

@@ -163,14 +163,15 @@ class DiT:
                 guidance: Optional[float] = None, txt_uncond: Optional[torch.Tensor] = None,
                 txt_len: Optional[Sequence[int]] = None,
                 txt_uncond_len: Optional[Sequence[int]] = None) -> torch.Tensor:
-        """FlowMatch-Euler loop (z-image-turbo-mnn "Scheduler"): n_steps forwards at
-        t = 1 - sigma'_i, each followed by zi_euler_step with sigma'_i -> sigma'_{i+1};
+        """FlowMatch-Euler loop (z-image-turbo-mnn "Scheduler"): n_steps forwards at the
+        library's timesteps (zi_timesteps: t_i = 1 - sigma'_i), each followed by zi_euler_step with sigma'_i -> sigma'_{i+1};
         with guidance and txt_uncond, the conditional and unconditional branches run
         as one batch-2 forward and are combined y_u + g (y_c - y_u).  txt_len /
         txt_uncond_len give the real lengths of padded prompts (see forward); the
         two branches' texts are padded to one length.  Returns the final latent (a
         new tensor; `latent` is left unchanged)."""
         sig = abi.sigmas(n_steps, shift)
+        ts = abi.timesteps(n_steps, shift)
         x = latent.clone()
         B = x.shape[0]
         cfg_mode = guidance is not None and txt_uncond is not None
@@ -191,7 +192,7 @@ class DiT:
             txt_all = txt
         x_in = torch.empty((2 * B,) + tuple(x.shape[1:]), dtype=torch.float32, device=x.device) if cfg_mode else x
         for i in range(n_steps):
-            tt.fill_(1.0 - sig[i])
+            tt.fill_(ts[i])
             if cfg_mode:
                 x_in[:B].copy_(x)
                 x_in[B:].copy_(x)
@@ -247,11 +248,12 @@ def denoise_cfg_split(latent: torch.Tensor, n_steps: int, shift: float, guidance
     if euler is None:
         euler = lambda x, yc, yu, g, s0, s1: euler_step(x, yc, yu, g, s0, s1)
     sig = abi.sigmas(n_steps, shift)
+    ts = abi.timesteps(n_steps, shift)
     x = latent.clone()
     t = torch.empty(x.shape[0], dtype=torch.float32, device=x.device)
     both = [torch.empty_like(x), torch.empty_like(x)]
     for i in range(n_steps):
-        t.fill_(1.0 - sig[i])
+        t.fill_(ts[i])
         y = forward(x, t)
         dist.all_gather(both, y.contiguous(), group=group)  # [conditional, unconditional]
         euler(x, both[0], both[1], float(guidance), sig[i], sig[i + 1])

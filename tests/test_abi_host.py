@@ -73,6 +73,24 @@ def test_sigmas_match_oracle(abi):
         np.testing.assert_allclose(abi.sigmas(n, shift), sch.sigmas(n, shift), rtol=0, atol=1e-15)
 
 
+def test_timesteps_match_oracle(abi):
+    """zi_timesteps gives the model timestep of every call, 1 - sigma'_i rounded to fp32 once
+    (z-image-turbo-mnn card, "Scheduler"), and nothing for the zero-sigma end point."""
+    for n, shift in ((8, 3.0), (1, 3.0), (30, 6.0), (4, 1.0)):
+        got = abi.timesteps(n, shift)
+        want = sch.timesteps(sch.sigmas(n, shift)).astype(np.float32)
+        assert len(got) == n
+        np.testing.assert_array_equal(np.array(got, dtype=np.float32), want)
+    # the 8-step Turbo schedule: t = 1 - 3k/(8 + 2k) for k = 8 .. 1, starting at 0 (pure noise)
+    got = abi.timesteps(8, 3.0)
+    assert got[0] == 0.0
+    np.testing.assert_allclose(got, [1.0 - 3.0 * k / (8.0 + 2.0 * k) for k in range(8, 0, -1)], rtol=0, atol=6e-8)
+    L = abi.lib()
+    assert L.zi_timesteps(0, 3.0, (ctypes.c_float * 1)()) == abi.ZI_ERR_ARG
+    assert L.zi_timesteps(4, 0.0, (ctypes.c_float * 4)()) == abi.ZI_ERR_ARG
+    assert L.zi_timesteps(4, 3.0, None) == abi.ZI_ERR_ARG
+
+
 def test_workspace_sizes(abi):
     c = abi.config_default()
     ws_block = abi.block_workspace_size(c, 1, 1152)

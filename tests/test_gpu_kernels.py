@@ -95,9 +95,10 @@ def test_pack_qkv_and_ffn_bit_exact(M):
                                    (4128, 3840, 3840), (2000, 2560, 1024), (4128, 3840, 64),
                                    (4128, 11520, 128), (19000, 256, 64)])
 def test_gemm_bf16(M, m, n, k):
-    """Covers single tiles, M tails, several waves, and ragged last waves that the
-    kernel cuts into 128 x 128 (4128 x 3840: 495 tiles) or 128 x 64 (19000 x 256:
-    149 tiles) sub-tiles."""
+    """Covers single tiles, M tails, several waves, and ragged last waves (4128 x 3840:
+    495 tiles = 3 x 148 + 51; 19000 x 256: 149 tiles).  The standalone entry point runs
+    every tile whole: it has no workspace for the fp32 partials of the K-split tail the
+    forward uses, which the block tests cover (test_full_width_block_split_tails_deterministic)."""
     abi, model = M
     a = zi.make_matrix((m, k), 3, 0)
     b = zi.make_matrix((n, k), 3, 1, std=0.05)

@@ -253,3 +253,106 @@ def test_pad_token_value_and_pad_features_do_not_leak():
     # without the key mask the pads would change the image tokens
     unmasked = ref.model_forward(lat, t, txt, ref.Weights(bits), d)
     assert np.abs(unmasked - base).max() > 1e-4
+
+
+# ------------------------------------------------------------------ timestep MLP and final layer
+# The timestep is passed to the model as 1 - sigma' (z-image-turbo-mnn card, "Scheduler") and
+# scaled by 1000 before a [cos, sin] sinusoid and the 256 -> 1024 -> SiLU -> 256 MLP (readings
+# of the same card's "Scheduler" and of the parameter count); the final layer is
+# LayerNorm(eps 1e-6, no affine) x (1 + Linear(SiLU(c))) -> Linear (H3ddle page, "What was
+# changed, and why": two small linears, final_layer.linear [64, 3840]).
+
+def _bits_of(arr):
+    """Exact small values (all representable in bf16) as bf16 bits."""
+    b = zi.f32_to_bf16_bits(np.asarray(arr, dtype=np.float32))
+    assert np.array_equal(zi.bf16_bits_to_f32(b), np.asarray(arr, dtype=np.float32))
+    return b
+
+
+def _silu(v):
+    return v / (1.0 + math.exp(-v))
+
+
+@pytest.mark.parametrize("t", [0.0, 0.3, 0.875])
+def test_t_embed_matches_brute_force(t):
+    d = zi.TINY
+    W = ref.Weights(_weights(d, 12))
+    got = ref.t_embed(np.array([t]), W)[0]
+    want = brute.t_embed_loop(t, W("t_embedder.linear1.weight").tolist(), W("t_embedder.linear1.bias").tolist(),
+                              W("t_embedder.linear2.weight").tolist(), W("t_embedder.linear2.bias").tolist())
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-13)
+
+
+def test_t_embed_closed_form():
+    """Selector weights make each output a hand-computable function of t:
+    c0 = 2 SiLU(cos(1000 t)), c1 = 2 SiLU(sin(1000 t)), c2 = 2 SiLU(cos(10 t))
+    (f_64 = 10000^(-1/2) = 1/100), c3 = 2 SiLU(sin(10 t)), c4 = SiLU(b1_4) with b1_4 = 0.5,
+    c5 = b2_5 = 0.25, every other output 0."""
+    d = zi.TINY
+    w1 = np.zeros((d.t_mid, d.t_freq), np.float32)
+    w1[0, 0] = w1[1, 128] = w1[2, 64] = w1[3, 192] = 1.0
+    b1 = np.zeros(d.t_mid, np.float32)
+    b1[4] = 0.5
+    w2 = np.zeros((d.ada_dim, d.t_mid), np.float32)
+    for i in range(4):
+        w2[i, i] = 2.0
+    w2[4, 4] = 1.0
+    b2 = np.zeros(d.ada_dim, np.float32)
+    b2[5] = 0.25
+    W = ref.Weights({"t_embedder.linear1.weight": _bits_of(w1), "t_embedder.linear1.bias": _bits_of(b1),
+                     "t_embedder.linear2.weight": _bits_of(w2), "t_embedder.linear2.bias": _bits_of(b2)})
+    for t in (0.0, 0.3, 0.875):
+        want = np.zeros(d.ada_dim)
+        want[0] = 2 * _silu(math.cos(1000 * t))
+        want[1] = 2 * _silu(math.sin(1000 * t))
+        want[2] = 2 * _silu(math.cos(10 * t))
+        want[3] = 2 * _silu(math.sin(10 * t))
+        want[4] = _silu(0.5)
+        want[5] = 0.25
+        np.testing.assert_allclose(ref.t_embed(np.array([t]), W)[0], want, rtol=1e-12, atol=1e-14)
+
+
+def test_final_layer_matches_brute_force():
+    d = zi.TINY
+    W = ref.Weights(_weights(d, 13))
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((3, d.dim)) * 0.7 + 0.2
+    c = rng.standard_normal(d.ada_dim) * 0.5
+    got = ref.final_layer(x, W, c)
+    args = [W(k).tolist() for k in ("final_layer.adaLN_modulation.weight", "final_layer.adaLN_modulation.bias",
+                                     "final_layer.linear.weight", "final_layer.linear.bias")]
+    for r in range(3):
+        np.testing.assert_allclose(got[r], brute.final_layer_loop(x[r].tolist(), c.tolist(), *args),
+                                   rtol=1e-11, atol=1e-13)
+
+
+def test_final_layer_closed_form():
+    """Row 0 alternates +-1 (mean 0, variance 1), row 1 is 3 +- 2 (mean 3, variance 4), so the
+    LayerNorm gives +-1/sqrt(1 + 1e-6) and +-1/sqrt(1 + 0.25e-6).  c = (1, -2, 0, ...) gives
+    SiLU(c) = (e/(1+e), -2/(1+e^2), 0, ...); adaLN weights 0.5 and 0.25 on those two inputs and
+    bias 0.125 make s = 0.5 SiLU(1) + 0.25 SiLU(-2) + 0.125 for every channel.  The final
+    linear picks channel 0 (output 0), channel 1 (output 1), their sum (output 2, which is 0)
+    and a bias of 0.75 (output 3)."""
+    d = zi.TINY
+    D, P = d.dim, d.patch_dim
+    sign = np.where(np.arange(D) % 2 == 0, 1.0, -1.0)
+    x = np.stack([sign, 3.0 + 2.0 * sign])
+    c = np.zeros(d.ada_dim)
+    c[0], c[1] = 1.0, -2.0
+    wa = np.zeros((D, d.ada_dim), np.float32)
+    wa[:, 0], wa[:, 1] = 0.5, 0.25
+    ba = np.full(D, 0.125, np.float32)
+    wf = np.zeros((P, D), np.float32)
+    wf[0, 0] = wf[1, 1] = wf[2, 0] = wf[2, 1] = 1.0
+    bf = np.zeros(P, np.float32)
+    bf[3] = 0.75
+    W = ref.Weights({"final_layer.adaLN_modulation.weight": _bits_of(wa),
+                     "final_layer.adaLN_modulation.bias": _bits_of(ba),
+                     "final_layer.linear.weight": _bits_of(wf), "final_layer.linear.bias": _bits_of(bf)})
+    s = 0.5 * (1.0 / (1.0 + math.exp(-1.0))) + 0.25 * (-2.0 / (1.0 + math.exp(2.0))) + 0.125
+    got = ref.final_layer(x, W, c)
+    for r, var in enumerate((1.0, 4.0)):
+        ln0 = 2.0 ** r / math.sqrt(var + 1e-6)  # |x - mean| is 1 in row 0 and 2 in row 1
+        want = np.zeros(P)
+        want[0], want[1], want[3] = ln0 * (1 + s), -ln0 * (1 + s), 0.75
+        np.testing.assert_allclose(got[r], want, rtol=1e-13, atol=1e-14)

@@ -74,6 +74,48 @@ def _block_without_post_norm(x, W, prefix, d, angles, c=None, return_parts=False
         ref.rms_norm = saved
 
 
+def _t_embed_no_scale(t, W):
+    e = ref.timestep_embedding(np.asarray(t, dtype=np.float64)).astype(W.dtype)  # t, not 1000 t
+    h = ref.silu(ref.linear(e, W("t_embedder.linear1.weight"), W("t_embedder.linear1.bias")))
+    return ref.linear(h, W("t_embedder.linear2.weight"), W("t_embedder.linear2.bias"))
+
+
+def _t_embed_silu_last(t, W):
+    e = ref.timestep_embedding(np.asarray(t, dtype=np.float64) * ref.T_SCALE).astype(W.dtype)
+    h = ref.linear(e, W("t_embedder.linear1.weight"), W("t_embedder.linear1.bias"))
+    return ref.silu(ref.linear(h, W("t_embedder.linear2.weight"), W("t_embedder.linear2.bias")))
+
+
+def _sinusoid_sin_first(t_in, width=256, max_period=10000.0):
+    e = ref.__dict__["_orig_timestep_embedding"](t_in, width, max_period)
+    return np.concatenate([e[:, width // 2:], e[:, :width // 2]], axis=-1)
+
+
+def _sinusoid_full_width_exponent(t_in, width=256, max_period=10000.0):
+    k = np.arange(width // 2, dtype=np.float64)
+    args = np.asarray(t_in, dtype=np.float64)[:, None] * np.exp(-np.log(max_period) * k / width)[None, :]
+    return np.concatenate([np.cos(args), np.sin(args)], axis=-1)
+
+
+def _final_layer_raw_c(x_img, W, c):
+    s = ref.linear(c, W("final_layer.adaLN_modulation.weight"), W("final_layer.adaLN_modulation.bias"))
+    return ref.linear(ref.layer_norm(x_img) * (1.0 + s), W("final_layer.linear.weight"), W("final_layer.linear.bias"))
+
+
+def _final_layer_scale_without_one(x_img, W, c):
+    s = ref.linear(ref.silu(c), W("final_layer.adaLN_modulation.weight"), W("final_layer.adaLN_modulation.bias"))
+    return ref.linear(ref.layer_norm(x_img) * s, W("final_layer.linear.weight"), W("final_layer.linear.bias"))
+
+
+def _final_layer_uncentred(x_img, W, c):
+    s = ref.linear(ref.silu(c), W("final_layer.adaLN_modulation.weight"), W("final_layer.adaLN_modulation.bias"))
+    y = x_img / np.sqrt(np.mean(x_img * x_img, axis=-1, keepdims=True) + ref.FINAL_EPS) * (1.0 + s)
+    return ref.linear(y, W("final_layer.linear.weight"), W("final_layer.linear.bias"))
+
+
+T_PINS = [tb.test_t_embed_closed_form, lambda: [tb.test_t_embed_matches_brute_force(t) for t in (0.3, 0.875)]]
+F_PINS = [tb.test_final_layer_closed_form, tb.test_final_layer_matches_brute_force]
+
 MUTATIONS = [
     ("apply_rope", _rope_half_split, [tp.test_rope_matches_explicit_rotation_matrix]),
     ("apply_rope", _rope_clockwise, [tp.test_rope_complex_product_convention]),
@@ -84,6 +126,13 @@ MUTATIONS = [
     ("patchify", _patchify_channel_slowest, [ts.test_patchify_matches_index_loop_and_roundtrips]),
     ("block_forward", _block_without_post_norm,
      [lambda: tb.test_post_norm_makes_output_rescaling_exact(True)]),
+    ("t_embed", _t_embed_no_scale, T_PINS),
+    ("t_embed", _t_embed_silu_last, T_PINS),
+    ("timestep_embedding", _sinusoid_sin_first, T_PINS + [tp.test_timestep_embedding_values]),
+    ("timestep_embedding", _sinusoid_full_width_exponent, T_PINS + [tp.test_timestep_embedding_values]),
+    ("final_layer", _final_layer_raw_c, F_PINS),
+    ("final_layer", _final_layer_scale_without_one, F_PINS),
+    ("final_layer", _final_layer_uncentred, F_PINS),
 ]
 
 
