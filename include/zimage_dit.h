@@ -288,8 +288,11 @@ ZI_API int zi_timesteps(int n_steps, double shift, float* h_t);
  *     rejected with ZI_ERR_SCRATCH_LIMIT before anything is enqueued (about 1,350
  *     tokens of batch x seq at Z-Image's full width).
  *   - The first call on each device looks up the scratch's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture on that device.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it for later
+ *     calls; make that first call before any stream capture on that device.
+ *     cudaDeviceReset destroys the array with the context, so the kept address
+ *     is stale afterwards: do not call this entry point on a device that was
+ *     reset earlier in the same process.
  *   - Every call on a device shares the one scratch array, and it keeps the last
  *     call's contents.  Nothing in it needs to start at zero (each call writes
  *     every scratch byte it reads), but calls whose GPU work overlaps -- on
@@ -350,6 +353,18 @@ ZI_API int zi_attention(const uint16_t* d_qkv, uint16_t* d_out, int batch, int s
 ZI_API int zi_attention_varlen(const uint16_t* d_qkv, uint16_t* d_out, int batch, int seq, int heads,
                                const int32_t* d_kv_len, zi_stream_t stream);
 
+/* Test hook for the attention softmax's second exponential: d_y[i] = 2^d_x[i] as the
+ * attention kernel computes it on the FMA pipe for 3 of every 8 score pairs (the rest
+ * go to the MUFU ex2 unit), so that its accuracy can be checked directly.  The method
+ * (the FMA-pipe exponential of FlashAttention-4, restated): x is clamped at -126;
+ * Cody-Waite split x = n + f with n = rint(x) (by adding and subtracting 1.5 * 2^23)
+ * and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients are a
+ * minimax fit of the relative error on [-1/2, 1/2] (Remez exchange); n is added to
+ * the result's exponent field.  Maximum relative error 7.5e-5 for x in (-126, 0],
+ * below the bf16 rounding the probabilities get next; x <= -126 (a masked key's
+ * -inf included) gives at most 2^-126.  d_x, d_y fp32 [n]; n == 0 enqueues nothing. */
+ZI_API int zi_exp2_poly(const float* d_x, float* d_y, size_t n, zi_stream_t stream);
+
 /* ---------------------------------------------------------------- launch profiling */
 
 /* Kernel identities reported by zi_profile_end. */
@@ -373,7 +388,8 @@ enum zi_kernel_kind {
   ZI_KERNEL_TEXT_PAD = 17,      /* cap_pad_token into padded text rows */
   ZI_KERNEL_SPLIT_CLEAR = 18,   /* zero the GEMM split-tail counters (once per forward) */
   ZI_KERNEL_QUANTIZE = 19,      /* zi_quantize_rows_e4m3 */
-  ZI_KERNEL_SELFTEST = 20       /* zi_watchdog_selftest */
+  ZI_KERNEL_SELFTEST = 20,      /* zi_watchdog_selftest */
+  ZI_KERNEL_EXP2_TEST = 21      /* zi_exp2_poly */
 };
 
 /* Start recording launch timings on this host thread: from the next kernel the

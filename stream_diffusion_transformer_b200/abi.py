@@ -85,6 +85,7 @@ _SIGS = {
     "zi_profile_begin": (c_int, [c_int]),
     "zi_profile_end": (c_int, [POINTER(c_float), POINTER(c_int), c_int, POINTER(c_int)]),
     "zi_watchdog_selftest": (c_int, [c_int, c_void_p]),
+    "zi_exp2_poly": (c_int, [c_void_p, c_void_p, c_size_t, c_void_p]),
     "zi_device_status": (c_int, [POINTER(c_int)]),
     "zi_clear_device_status": (c_int, []),
 }
@@ -175,6 +176,7 @@ KERNEL_NAMES = {
     5: "gemm_ffn_down", 6: "post_norm_residual", 7: "pre_norm", 8: "adaln_gemv", 9: "timestep_mlp",
     10: "rope_table", 11: "positions", 12: "patchify", 13: "gemm_embed", 14: "gemm_final_unpatchify",
     15: "euler", 16: "gemm", 17: "text_pad", 18: "split_clear", 19: "quantize_e4m3", 20: "watchdog_selftest",
+    21: "exp2_poly_test",
 }
 
 

@@ -543,6 +543,18 @@ int run_rope(const zi_config& cfg, const int32_t* pos, int n, float2* out, cudaS
   return launched(ZI_KERNEL_ROPE, st);
 }
 
+// Elementwise 2^x through the attention softmax's FMA-pipe exponential (exp2_poly_pair),
+// for the test hook zi_exp2_poly.
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, size_t n) {
+  const size_t i = 2 * (size_t(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  float e0, e1;
+  exp2_poly_pair(x[i], two ? x[i + 1] : 0.f, e0, e1);
+  y[i] = e0;
+  if (two) y[i + 1] = e1;
+}
+
 // ---------------------------------------------------------------- fixed scratch
 // Scratch of zi_block_forward_noalloc: a file-scope device array, so the entry
 // point needs no caller workspace and allocates nothing.  Host code must not use
@@ -1231,6 +1243,18 @@ int zi_watchdog_selftest(int limit_us, zi_stream_t stream) {
   prof_pre(st);
   watchdog_selftest_kernel<<<1, 32, 0, st>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
   return launched(ZI_KERNEL_SELFTEST, st);
+}
+
+int zi_exp2_poly(const float* d_x, float* d_y, size_t n, zi_stream_t stream) {
+  if (n == 0) return ZI_OK;
+  if (!d_x || !d_y) return ZI_ERR_ARG;
+  DevInfo* dev;
+  ZI_TRY(current_device(&dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t threads = (n + 1) / 2;
+  prof_pre(st);
+  exp2_poly_kernel<<<unsigned((threads + 255) / 256), 256, 0, st>>>(d_x, d_y, n);
+  return launched(ZI_KERNEL_EXP2_TEST, st);
 }
 
 int zi_device_status(int* h_code) {
