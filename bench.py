@@ -392,6 +392,36 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     h2d = h_lat.numel() * 4 + h_txt.numel() * 2 + h_t.numel() * 4
     d2h = h_out.numel() * 4
 
+    # ---- the same forward with e4m3 block projections (the quantised variants the pages
+    # are about), on the resident bf16 weights: same inputs, same timing rules
+    e4m3 = {}
+    if not args.no_e4m3:
+        for mode, name, what in ((True, "e4m3_qkv_ffn_up", "e4m3 QKV and FFN w1|w3 projections, bf16 elsewhere"),
+                                 ("all", "e4m3_all_projections", "e4m3 QKV, output, FFN w1|w3 and w2 projections")):
+            dit8 = dit.with_e4m3(mode)
+            for _ in range(args.warmup):
+                dit8.forward(lat, tt, txt, out)
+            torch.cuda.synchronize()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(local_rank) as clk8:
+                barrier()
+                torch.cuda.synchronize()
+                f0.record(stream)
+                for _ in range(args.steps):
+                    dit8.forward(lat, tt, txt, out)
+                f1.record(stream)
+                torch.cuda.synchronize()
+                barrier()
+            ms8 = max_over_ranks(f0.elapsed_time(f1), world, dev)
+            e4m3[name] = {"value": flops * world * args.steps / (ms8 * 1e-3) / 1e12, "unit": "TFLOP/s",
+                          "ms_per_step": ms8 / args.steps, "steps": args.steps, "warmup": args.warmup,
+                          "dtype": what, "flops": "counted as for the bf16 forward",
+                          "output_finite": bool(torch.isfinite(out).all().item()), "clocks": clk8.summary()}
+            del dit8
+            torch.cuda.empty_cache()
+        if abi.device_status() != 0:
+            raise RuntimeError("device pipeline timeout during the e4m3 forwards")
+
     if rank != 0:
         return
 
@@ -478,6 +508,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps},
         "clocks": clk,
         "output_finite": out_finite,
+        "e4m3_forwards": e4m3,
         "published_context": {"ms": 22500.0, "hardware": "Apple M1 Pro", "precision": "int8 ConvRot",
                               "source": "Z-Image-Turbo repackaged for H3ddle, Measured performance"},
     }
@@ -675,6 +706,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e4m3", action="store_true", help="skip the e4m3 forwards after the headline timing")
     ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8", "fp8all", "oracle"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
                          "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens; "

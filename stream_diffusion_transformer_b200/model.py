@@ -102,6 +102,12 @@ class DeviceBlock:
             self.t["w_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.weight"], device)
             self.t["b_ada"] = upload_bits(bits[f"{prefix}.adaLN_modulation.bias"], device)
         self.modulated = modulated
+        self._finish(fp8)
+
+    BF16_FIELDS = ("w_qkv", "w_out", "w13", "w2", "g_attn1", "g_attn2", "g_ffn1", "g_ffn2", "g_q", "g_k",
+                   "w_ada", "b_ada")
+
+    def _finish(self, fp8):
         if fp8:
             groups = [("w_qkv", "w_qkv8", "s_qkv"), ("w13", "w13_8", "s_13")]
             if fp8 == "all":
@@ -111,6 +117,15 @@ class DeviceBlock:
         self.fp8 = fp8
         self.struct = abi.ZiBlockWeights(**{f: (self.t[f].data_ptr() if f in self.t else None)
                                             for f in abi.BLOCK_FIELDS})
+
+    def with_e4m3(self, fp8=True) -> "DeviceBlock":
+        """The same block sharing these bf16 tensors, with e4m3 codes made from them (see the
+        class docstring for fp8)."""
+        b = DeviceBlock.__new__(DeviceBlock)
+        b.t = {k: v for k, v in self.t.items() if k in self.BF16_FIELDS}
+        b.modulated = self.modulated
+        b._finish(fp8)
+        return b
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in self.t.values())
@@ -137,6 +152,9 @@ class DiT:
                                 False, self.device, fp8) for i in range(cfg.n_ctx)]
         self.main = [DeviceBlock(cfg, f"layers.{i}", fetch(block_keys(f"layers.{i}", True)), True, self.device, fp8)
                      for i in range(cfg.n_main)]
+        self._bind()
+
+    def _bind(self):
         self._noise_arr = (abi.ZiBlockWeights * max(1, len(self.noise)))(*[b.struct for b in self.noise])
         self._ctx_arr = (abi.ZiBlockWeights * max(1, len(self.ctx)))(*[b.struct for b in self.ctx])
         self._main_arr = (abi.ZiBlockWeights * len(self.main))(*[b.struct for b in self.main])
@@ -147,6 +165,18 @@ class DiT:
         self.weights.ctx = ctypes.cast(self._ctx_arr, ctypes.POINTER(abi.ZiBlockWeights))
         self.weights.main = ctypes.cast(self._main_arr, ctypes.POINTER(abi.ZiBlockWeights))
         self._ws: Dict[tuple, torch.Tensor] = {}
+
+    def with_e4m3(self, fp8=True) -> "DiT":
+        """This transformer with its block projections in e4m3 (fp8=True: QKV and FFN w1|w3;
+        "all": every block projection), sharing the resident bf16 weights: only the e4m3
+        codes and their per-row scales are new (zi_quantize_rows_e4m3 on the device)."""
+        other = DiT.__new__(DiT)
+        other.cfg, other.device, other.top, other.fp8 = self.cfg, self.device, self.top, fp8
+        other.noise = [b.with_e4m3(fp8) for b in self.noise]
+        other.ctx = [b.with_e4m3(fp8) for b in self.ctx]
+        other.main = [b.with_e4m3(fp8) for b in self.main]
+        other._bind()
+        return other
 
     def nbytes(self) -> int:
         n = sum(t.numel() * t.element_size() for t in self.top.values())
@@ -164,8 +194,8 @@ class DiT:
                 txt_len: Optional[Sequence[int]] = None,
                 txt_uncond_len: Optional[Sequence[int]] = None) -> torch.Tensor:
         """FlowMatch-Euler loop (z-image-turbo-mnn "Scheduler"): n_steps forwards at the
-        library's timesteps (zi_timesteps: t_i = 1 - sigma'_i), each followed by zi_euler_step with sigma'_i -> sigma'_{i+1};
-        with guidance and txt_uncond, the conditional and unconditional branches run
+        library's timesteps (zi_timesteps: t_i = 1 - sigma'_i), each followed by
+        zi_euler_step with sigma'_i -> sigma'_{i+1}; with guidance and txt_uncond, the conditional and unconditional branches run
         as one batch-2 forward and are combined y_u + g (y_c - y_u).  txt_len /
         txt_uncond_len give the real lengths of padded prompts (see forward); the
         two branches' texts are padded to one length.  Returns the final latent (a
