@@ -360,9 +360,10 @@ ZI_API int zi_attention_varlen(const uint16_t* d_qkv, uint16_t* d_out, int batch
  * Cody-Waite split x = n + f with n = rint(x) (by adding and subtracting 1.5 * 2^23)
  * and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients are a
  * minimax fit of the relative error on [-1/2, 1/2] (Remez exchange); n is added to
- * the result's exponent field.  Maximum relative error 7.5e-5 for x in (-126, 0],
- * below the bf16 rounding the probabilities get next; x <= -126 (a masked key's
- * -inf included) gives at most 2^-126.  d_x, d_y fp32 [n]; n == 0 enqueues nothing. */
+ * the result's exponent field.  Maximum relative error 7.5e-5 for x in [-125, 0],
+ * below the bf16 rounding the probabilities get next; below -125 (where the result
+ * can fall into the denormal range; a masked key's -inf included) it gives a value
+ * in [0, 2^-124].  d_x, d_y fp32 [n]; n == 0 enqueues nothing. */
 ZI_API int zi_exp2_poly(const float* d_x, float* d_y, size_t n, zi_stream_t stream);
 
 /* ---------------------------------------------------------------- launch profiling */

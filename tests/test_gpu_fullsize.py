@@ -24,6 +24,7 @@ tokens, all 34 blocks at full width) is also compared end to end with the
 fp64 oracle.
 """
 import os
+import time
 from collections.abc import Mapping
 
 import numpy as np
@@ -213,7 +214,10 @@ def test_full_stack_4128_tokens_end_to_end(run):
     d, s_img = run["d"], run["s_img"]
     W = ref.Weights(LazyBits(d, SEED, max(1, min(16, os.cpu_count() or 1))), dtype=np.float32)
     trace = []
+    t0 = time.perf_counter()
     want = ref.model_forward(run["lat"], run["t"], zi.bf16_bits_to_f32(run["txt"]), W, d, trace=trace)
+    print(f"[oracle] full 4,128-token forward (fp32 NumPy, {os.cpu_count()} host CPUs): "
+          f"{time.perf_counter() - t0:.1f} s including weight generation")
     order = ([f"noise_refiner.{i}" for i in range(d.n_noise)] + [f"context_refiner.{i}" for i in range(d.n_ctx)]
              + [f"layers.{i}" for i in range(d.n_main)])
     worst = 1.0
