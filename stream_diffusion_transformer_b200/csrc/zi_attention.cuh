@@ -140,8 +140,9 @@ ZI_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
 // MUFU): Cody-Waite split x = n + f with n = rint(x) (the 1.5 * 2^23 rounding
 // trick), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients were
 // fitted here by the Remez exchange algorithm on the relative error (max
-// relative error 7.5e-5, far below the bf16 rounding P gets next); n is added
-// to the exponent field.  x is clamped at -126 so the result stays normal.
+// relative error 7.5e-5 on [-125, 0], far below the bf16 rounding P gets next); n
+// is added to the exponent field.  x is clamped at -126; below -125 the result may
+// be denormal and is at most 2^-124 (zero at P's precision against a row max of 1).
 ZI_DEV void exp2_poly_pair(float x0, float x1, float& e0, float& e1) {
   x0 = fmaxf(x0, -126.0f);
   x1 = fmaxf(x1, -126.0f);
