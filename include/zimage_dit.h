@@ -324,6 +324,14 @@ ZI_API int zi_rope_table(const zi_config* cfg, const int32_t* d_pos, int n, floa
 ZI_API int zi_gemm_bf16(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k,
                         zi_stream_t stream);
 
+/* zi_gemm_bf16 on CTA pairs: two CTAs of a cluster on two SMs compute each 256 x 256
+ * output tile with one tcgen05 cta_group::2 instruction stream (A rows split between
+ * them, B split along N), so each SM stages 32 KB of operands per 64-deep k-block
+ * instead of 48 KB.  Same arguments, restrictions and result as zi_gemm_bf16; the
+ * forward picks per projection whichever of the two kernels suits its shape. */
+ZI_API int zi_gemm_bf16_pair(const uint16_t* d_a, const uint16_t* d_b, uint16_t* d_c, int m, int n, int k,
+                             zi_stream_t stream);
+
 /* Per-row e4m3 quantisation (OCP e4m3: bias 7, 3 mantissa bits, max 448):
  *   s[r] = amax_r / 448 (fp32), q[r][k] = e4m3(x[r][k] * (448 / amax_r)), the
  *   product formed in fp32, rounded to nearest even, saturating at +-448; a row of

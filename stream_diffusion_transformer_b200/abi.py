@@ -78,6 +78,7 @@ _SIGS = {
     "zi_positions": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),
     "zi_rope_table": (c_int, [POINTER(ZiConfig), c_void_p, c_int, c_void_p, c_void_p]),
     "zi_gemm_bf16": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "zi_gemm_bf16_pair": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_attention": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "zi_quantize_rows_e4m3": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "zi_gemm_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),

@@ -14,9 +14,8 @@
 //               one half of the tile's columns): tcgen05.ld TMEM -> registers ->
 //               fused math -> global
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the epilogue
-// of tile i overlaps the main loop of tile i + 1.  Tiles are walked along the
-// shorter output dimension first (tile_origin), so that CTAs running at the same
-// time share the larger operand's tiles through L2.
+// of tile i overlaps the main loop of tile i + 1.  Tiles are walked in groups that
+// keep one operand's panels in L2 while the other is swept (tile_origin).
 #pragma once
 #include "zi_common.cuh"
 
@@ -267,28 +266,60 @@ struct TailSched {
   int tail_items;  // CTAs [0, tail_items) each run piece c % s of tile dp_tiles + c / s
   int kb;          // k-blocks per tile
   int num_n;       // N tiles
-  int n_fast;      // tile index walks N fastest (else M fastest)
+  int group;       // tiles per group along the grouped dimension (see tile_origin)
+  int group_n;     // 1: groups of N tiles (B panels held in L2), 0: groups of M tiles
 };
 
-// Tile t covers rows [m0, m0 + BM) and columns [n0, n0 + BN).  The index walks the
-// shorter dimension of the output fastest, so that the CTAs running at the same
-// time share the tiles of the larger operand through L2 while the smaller one stays
-// resident: M-fastest when N > M (the weight is the larger operand), N-fastest when
-// M > N (then the activation is, e.g. FFN down's 4,128 x 10,240 input, which would
-// otherwise be re-read from DRAM for every wave).
+// Tile t covers rows [m0, m0 + BM) and columns [n0, n0 + BN).  Tiles are walked in
+// groups: `group` M tiles (their A panels) swept over every N tile with M fastest
+// inside the group, or `group` N tiles swept over every M tile with N fastest.  The
+// CTAs running at the same time then read a few panels of the swept operand while
+// the group's panels stay in L2 for the whole sweep, so from DRAM the grouped operand
+// is read once and the swept one once per group (choose_raster picks the side and
+// the group size from the operands' sizes).
 template <int BM, int BN>
 ZI_DEV void tile_origin(const TailSched& s, int num_m, int tile, int& m0, int& n0) {
-  if (s.n_fast) {
-    m0 = (tile / s.num_n) * BM;
-    n0 = (tile % s.num_n) * BN;
+  if (s.group_n) {
+    const int per = s.group * num_m;
+    const int g = tile / per, r = tile - g * per;
+    const int cols = min(s.group, s.num_n - g * s.group);
+    n0 = (g * s.group + r % cols) * BN;
+    m0 = (r / cols) * BM;
   } else {
-    m0 = (tile % num_m) * BM;
-    n0 = (tile / num_m) * BN;
+    const int per = s.group * s.num_n;
+    const int g = tile / per, r = tile - g * per;
+    const int rows = min(s.group, num_m - g * s.group);
+    m0 = (g * s.group + r % rows) * BM;
+    n0 = (r / rows) * BN;
   }
 }
 
-inline TailSched make_tail_sched(int tiles, int grid, int kb, bool can_split, int num_n, bool n_fast) {
-  TailSched s{grid, tiles, 1, 0, kb, num_n, n_fast ? 1 : 0};
+// Bytes of one operand's panels a group may keep in L2 (about 45% of the 126 MB, so
+// the swept operand's tiles, the output and other traffic still fit beside them).
+constexpr double kRasterL2Budget = 56.0e6;
+
+// Picks the grouped side and group size with the fewest DRAM bytes: grouping M tiles
+// reads A once and B once per group, grouping N tiles the reverse.  a_panel / b_panel:
+// bytes of one M tile's rows of A / one N tile's rows of B over the whole K.
+inline void choose_raster(int num_m, int num_n, double a_panel, double b_panel, int& group, int& group_n) {
+  auto fit = [](double panel, int n) {
+    int g = panel > 0 ? int(kRasterL2Budget / panel) : n;
+    return g < 1 ? 1 : (g > n ? n : g);
+  };
+  const int gm = fit(a_panel, num_m), gn = fit(b_panel, num_n);
+  const double tm = num_m * a_panel + double((num_m + gm - 1) / gm) * num_n * b_panel;
+  const double tn = num_n * b_panel + double((num_n + gn - 1) / gn) * num_m * a_panel;
+  if (tn < tm) {
+    group = gn;
+    group_n = 1;
+  } else {
+    group = gm;
+    group_n = 0;
+  }
+}
+
+inline TailSched make_tail_sched(int tiles, int grid, int kb, bool can_split, int num_n, int group, int group_n) {
+  TailSched s{grid, tiles, 1, 0, kb, num_n, group, group_n};
   const int rounds = tiles / grid, rest = tiles - rounds * grid;
   if (!can_split || rest == 0 || grid > kSplitSlots) return s;
   int f = grid / rest;
@@ -579,6 +610,279 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
   }
+}
+
+// ------------------------------------------------------------------ CTA-pair GEMM
+// The same product on CTA pairs (tcgen05 cta_group::2): a pair computes a 256 x 256
+// output tile, each CTA loading its own 128 rows of A and its own half (128 rows) of
+// the tile's B, so a CTA moves 32 KB of operands per 64-deep (bf16) k-block instead of
+// the 48 KB a 128 x 256 tile on one SM needs; CTA 0 issues M = 256 MMAs for both SMs,
+// each CTA's TMEM holds its 128 rows x 256 columns (double-buffered), and each CTA's
+// epilogue writes its own rows with the same fused epilogues.  Work units are the
+// pair's tiles, walked like the single-CTA kernel's (tile_origin with BM = 256); a
+// ragged last wave is cut along K the same way, each CTA keeping its own partials
+// and counter for its 128 rows.
+template <int STAGES>
+struct PairSmem {
+  static constexpr uint32_t kABytes = 128u * 128u;  // 128 rows x 128 bytes of K
+  static constexpr uint32_t kBBytes = 128u * 128u;  // this CTA's 128 rows of the 256-row B tile
+  static constexpr uint32_t kStage = kABytes + kBBytes;
+  static constexpr uint32_t kBarOff = STAGES * kStage;
+  static constexpr uint32_t kBytes = kBarOff + 256u + 1024u;
+};
+
+template <int STAGES, int EPI, bool F8>
+ZI_DEV void gemm_pair_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, const EpiParams& ep,
+                           const TailSched& sched, const SplitScratch& sk) {
+  using L = PairSmem<STAGES>;
+  constexpr int BN = 256, BM = 256, BK = F8 ? 128 : 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);  // CTA 0: both CTAs' stage s loaded
+  uint64_t* empty = full + STAGES;     // each CTA: its stage s consumed by the pair's MMAs
+  uint64_t* tfull = empty + STAGES;    // each CTA: accumulator complete
+  uint64_t* tempty = tfull + 2;        // CTA 0: both CTAs' epilogues drained the accumulator
+  uint64_t* drain = tempty + 2;
+  uint64_t* ebar = drain + 1;          // this CTA's epilogue warps' own barrier (split tail)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int unit = blockIdx.x >> 1;  // the pair's index in the work schedule
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kEpiWarps);  // one arrival per epilogue warp of each CTA
+    }
+    mbar_init(drain, 1);
+    mbar_init(ebar, 32 * kEpiWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated before any remote access
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // an earlier kernel timed out: every role skips its work, both CTAs still meet at the end
+  const bool err = device_error_set();
+
+  const int num_m = (M + BM - 1) / BM;
+  WorkItem wi;
+
+  if (err) {
+  } else if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      WorkWalker walk(sched, unit);
+      while (walk.next(wi)) {
+        int m0, n0;
+        tile_origin<BM, BN>(sched, num_m, wi.tile, m0, n0);
+        bool ok = true;
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * L::kStage;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * L::kStage);
+          tma_load_2d_pair(sa, &tmA, &full[s], kb * BK, m0 + 128 * int(rank));
+          tma_load_2d_pair(sa + L::kABytes, &tmB, &full[s], kb * BK, n0 + 128 * int(rank));
+          ++it;
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+      WorkWalker walk(sched, unit);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(256, BN) : idesc_bf16_f32(256, BN, false, false);
+      while (ok && walk.next(wi)) {
+        const int acc = local & 1;
+        const uint32_t u = uint32_t(local) >> 1;
+        ++local;
+        if (!mbar_wait(&tempty[acc], (u & 1u) ^ 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(acc * BN);
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&full[s], r & 1u, abort_flag, ZI_DEVERR_TIMEOUT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * L::kStage);
+          const uint32_t b_addr = a_addr + L::kABytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per MMA
+            const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16), bd = smem_desc_sw128(b_addr + k * 32, 16);
+            const uint32_t acc_in = (kb != wi.kb0 || k != 0) ? 1u : 0u;
+            if constexpr (F8) {
+              tc_mma2_f8(d, ad, bd, idesc, acc_in);
+            } else {
+              tc_mma2(d, ad, bd, idesc, acc_in);
+            }
+          }
+          tc_commit_pair(&empty[s]);
+          ++it;
+        }
+        if (ok) tc_commit_pair(&tfull[acc]);
+      }
+      if (!ok) {
+        tc_commit_pair_local(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never, ZI_DEVERR_TIMEOUT_DRAIN);
+      }
+    }
+  } else {
+    const int q = warp & 3;             // this warp's TMEM lane quarter
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns
+    const int row_in_tile = q * 32 + lane;
+    int local = 0;
+    uint32_t ephase = 0;
+    auto epi_sync = [&]() -> bool {  // this CTA's epilogue threads meet (bounded wait)
+      mbar_arrive(ebar);
+      const bool r = mbar_wait(ebar, ephase, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE);
+      ephase ^= 1u;
+      return r;
+    };
+    WorkWalker walk(sched, unit);
+    while (walk.next(wi)) {
+      const int acc = local & 1;
+      const uint32_t u = uint32_t(local) >> 1;
+      ++local;
+      if (!mbar_wait(&tfull[acc], u & 1u, abort_flag, ZI_DEVERR_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      int m0, n0;
+      tile_origin<BM, BN>(sched, num_m, wi.tile, m0, n0);
+      const int row = m0 + 128 * int(rank) + row_in_tile;
+      const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+      bool finish = true;
+      if (wi.piece >= 0) {
+        // A piece of a split tile: publish this CTA's partial, finish only if last
+        // among the pieces' CTAs of the same rank.
+        const int slot0 = 2 * (unit - wi.piece) + int(rank);  // piece 0's slot for this rank; piece j at slot0 + 2 j
+        float4* mine = sk.partials + size_t(blockIdx.x) * (32 * BN) + row_in_tile;
+        for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(tb + c * 32, v);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            __stcg(mine + size_t(c * 8 + k) * 128,
+                   make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                               __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+        }
+        __threadfence();
+        if (!epi_sync()) break;
+        if (threadIdx.x == 64) {
+          const int t = 2 * (wi.tile - sched.dp_tiles) + int(rank);
+          const int old = atomicAdd(&sk.counters[t], 1);
+          const bool last = old == sched.tail_s - 1;
+          if (last) sk.counters[t] = 0;  // ready for the next launch
+          *last_flag = last ? 1 : 0;
+        }
+        if (!epi_sync()) break;
+        finish = *last_flag != 0;
+        if (finish) {
+          __threadfence();
+          for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+            uint32_t v[32];
+            tmem_ld32_sync(tb + c * 32, v);
+            float4 tot[8];
+            for (int j = 0; j < sched.tail_s; ++j) {
+              float4 pj[8];
+              if (j == wi.piece) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                  pj[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                      __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+              } else {
+                const float4* src =
+                    sk.partials + size_t(slot0 + 2 * j) * (32 * BN) + size_t(c * 8) * 128 + row_in_tile;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) pj[k] = __ldcg(src + size_t(k) * 128);
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                if (j == 0) {
+                  tot[k] = pj[k];
+                } else {
+                  tot[k].x += pj[k].x;
+                  tot[k].y += pj[k].y;
+                  tot[k].z += pj[k].z;
+                  tot[k].w += pj[k].w;
+                }
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              v[4 * k] = __float_as_uint(tot[k].x);
+              v[4 * k + 1] = __float_as_uint(tot[k].y);
+              v[4 * k + 2] = __float_as_uint(tot[k].z);
+              v[4 * k + 3] = __float_as_uint(tot[k].w);
+            }
+            tmem_st32(tb + c * 32, v);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (finish) gemm_epilogue<EPI, BN, F8>(tb, row, row < M, n0, half, ep);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_leader(&tempty[acc]);
+    }
+  }
+
+  if (*abort_flag) {  // an aborted pipeline: let copies already issued land before the pair leaves
+    const unsigned long long t0 = globaltimer();
+    while (globaltimer() - t0 < 200000ull) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA frees TMEM or exits while the pair's MMAs or copies may use it
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512) : "memory");
+  }
+}
+
+template <int STAGES, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                          EpiParams ep, TailSched sched, SplitScratch sk) {
+  gemm_pair_body<STAGES, EPI, false>(tmA, tmB, M, ep, sched, sk);
+}
+
+template <int STAGES, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_e4m3_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                          EpiParams ep, TailSched sched, SplitScratch sk) {
+  gemm_pair_body<STAGES, EPI, true>(tmA, tmB, M, ep, sched, sk);
 }
 
 template <int BN, int STAGES, int EPI>

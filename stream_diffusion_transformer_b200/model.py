@@ -366,13 +366,13 @@ def rope_table(cfg: abi.ZiConfig, pos: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def gemm(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """a bf16 [M, K] @ b bf16 [N, K]^T -> bf16 [M, N]."""
+def gemm(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None, pair: bool = False) -> torch.Tensor:
+    """a bf16 [M, K] @ b bf16 [N, K]^T -> bf16 [M, N]; pair=True runs it on CTA pairs (zi_gemm_bf16_pair)."""
     M, K = a.shape
     N = b.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
-    abi.call("zi_gemm_bf16", _p(a), _p(b), _p(out), M, N, K, _stream())
+    abi.call("zi_gemm_bf16_pair" if pair else "zi_gemm_bf16", _p(a), _p(b), _p(out), M, N, K, _stream())
     return out
 
 

@@ -110,6 +110,29 @@ def test_gemm_bf16(M, m, n, k):
     assert np.abs(got - want).max() <= 1e-2 * np.abs(want).max() + 1e-6
 
 
+@pytest.mark.parametrize("m,n,k", [(1, 256, 64), (96, 768, 256), (255, 256, 128), (257, 512, 192),
+                                   (300, 1536, 256), (1152, 3840, 3840), (4128, 3840, 3840),
+                                   (4128, 20480, 640), (2000, 2560, 1024), (4128, 3840, 64),
+                                   (19000, 256, 64), (33792, 768, 128)])
+def test_gemm_bf16_pair(M, m, n, k):
+    """The CTA-pair kernel (256 x 256 tiles, B split across the two SMs): single tiles,
+    rows past M in either CTA of the last tile pair (255, 257, 4128 rows), fewer tiles than
+    pairs, several waves, and exact multiples of 256 rows (33,792, the CFG size)."""
+    abi, model = M
+    a = zi.make_matrix((m, k), 6, 0)
+    b = zi.make_matrix((n, k), 6, 1, std=0.05)
+    c = model.gemm(dev_bits(a), dev_bits(b), pair=True)
+    torch.cuda.synchronize()
+    want = bits_f64(a) @ bits_f64(b).T
+    got = host_f64(c)
+    assert rel_l2(got, want) <= 4e-3
+    assert np.abs(got - want).max() <= 1e-2 * np.abs(want).max() + 1e-6
+    # the single-CTA kernel accumulates every output in the same K order: identical bits
+    c1 = model.gemm(dev_bits(a), dev_bits(b))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(c.view(torch.int16).cpu().numpy(), c1.view(torch.int16).cpu().numpy())
+
+
 @pytest.mark.parametrize("batch,seq,heads", [(1, 96, 2), (1, 128, 1), (2, 200, 2), (1, 1152, 4), (1, 33, 3)])
 def test_attention(M, batch, seq, heads):
     abi, model = M
