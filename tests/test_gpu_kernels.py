@@ -93,10 +93,14 @@ def test_pack_qkv_and_ffn_bit_exact(M):
 @pytest.mark.parametrize("m,n,k", [(1, 256, 64), (96, 768, 256), (127, 256, 128), (129, 512, 192),
                                    (300, 1536, 256), (1152, 3840, 3840), (4128, 1280, 640),
                                    (4128, 3840, 3840), (2000, 2560, 1024), (4128, 3840, 64),
-                                   (4128, 11520, 128), (19000, 256, 64)])
+                                   (4128, 11520, 128), (19000, 256, 64), (4128, 3840, 10240),
+                                   (8192, 3584, 16384), (32768, 4096, 8192)])
 def test_gemm_bf16(M, m, n, k):
     """Covers single tiles, M tails, several waves, and ragged last waves (4128 x 3840:
-    495 tiles = 3 x 148 + 51; 19000 x 256: 149 tiles).  The standalone entry point runs
+    495 tiles = 3 x 148 + 51; 19000 x 256: 149 tiles), and the grouped tile walk with a
+    partial last group: 4128 x 3840 x 10240 walks groups of 21 and 12 row tiles,
+    8192 x 3584 x 16384 groups of 13 row tiles (the last 12), 32768 x 4096 x 8192 groups
+    of 13 and 3 column tiles.  The standalone entry point runs
     every tile whole: it has no workspace for the fp32 partials of the K-split tail the
     forward uses, which the block tests cover (test_full_width_block_split_tails_deterministic)."""
     abi, model = M
@@ -113,11 +117,14 @@ def test_gemm_bf16(M, m, n, k):
 @pytest.mark.parametrize("m,n,k", [(1, 256, 64), (96, 768, 256), (255, 256, 128), (257, 512, 192),
                                    (300, 1536, 256), (1152, 3840, 3840), (4128, 3840, 3840),
                                    (4128, 20480, 640), (2000, 2560, 1024), (4128, 3840, 64),
-                                   (19000, 256, 64), (33792, 768, 128)])
+                                   (19000, 256, 64), (33792, 768, 128), (4128, 3840, 10240),
+                                   (8192, 3584, 16384)])
 def test_gemm_bf16_pair(M, m, n, k):
     """The CTA-pair kernel (256 x 256 tiles, B split across the two SMs): single tiles,
     rows past M in either CTA of the last tile pair (255, 257, 4128 rows), fewer tiles than
-    pairs, several waves, and exact multiples of 256 rows (33,792, the CFG size)."""
+    pairs, several waves, exact multiples of 256 rows (33,792, the CFG size), and grouped
+    tile walks with a partial last group (4128 x 3840 x 10240: 10 + 7 row tiles;
+    8192 x 3584 x 16384: 6 + 6 + 2 column tiles)."""
     abi, model = M
     a = zi.make_matrix((m, k), 6, 0)
     b = zi.make_matrix((n, k), 6, 1, std=0.05)
