@@ -5,14 +5,18 @@
 // checkpoint's own [out, in] orientation, which is exactly the K-major operand
 // tcgen05 wants, so weights are used as stored.
 //
-// One CTA per SM, 10 warps:
-//   warp 0      TMA producer: a 128-row A tile + a BN-row B tile of 128 bytes of K
-//               per stage (64 bf16 or 128 e4m3), 128-byte swizzle, STAGES-deep ring
+// Two kernels share one structure, 10 warps per CTA:
+//   warp 0      TMA producer: a 128-row A tile + a B tile of 128 bytes of K per
+//               stage (64 bf16 or 128 e4m3), 128-byte swizzle, STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//               (M = 128, N = BN, 32 bytes of K per instruction; fp32 accumulator in TMEM)
+//               (32 bytes of K per instruction; fp32 accumulator in TMEM)
 //   warps 2..9  epilogue in two groups of four (each covers all 128 TMEM lanes and
 //               one half of the tile's columns): tcgen05.ld TMEM -> registers ->
 //               fused math -> global
+// gemm_tn_body: one CTA per SM computes 128 x BN tiles (M = 128 MMAs, a BN-row B
+// tile per stage).  gemm_pair_body: a cluster of two CTAs on two SMs computes
+// 256 x 256 tiles with cta_group::2 MMAs (M = 256) issued by CTA 0; each CTA stages
+// its own 128 rows of A and its 128-row half of B (see the comment above it).
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the epilogue
 // of tile i overlaps the main loop of tile i + 1.  Tiles are walked in groups that
 // keep one operand's panels in L2 while the other is swept (tile_origin).
