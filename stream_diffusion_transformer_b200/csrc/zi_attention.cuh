@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -451,7 +451,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tmem_st32(s_addr + 32, &pw[32]);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_full[t]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[t]);  // for the whole warp: its stores are complete
       }
       ok = ok && mbar_wait(&pv_done[t], uint32_t(nj - 1) & 1u, abort_flag, ZI_DEVERR_TIMEOUT_SOFTMAX);
       if (ok) tc_fence_after();
