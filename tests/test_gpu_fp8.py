@@ -197,3 +197,26 @@ def test_full_width_model_all_e4m3():
     bf16 = ref.model_forward(*args)
     r = np.linalg.norm(want - bf16) / np.linalg.norm(bf16)
     print(f"[fp8] oracle e4m3-all vs bf16 model output: rel-L2 {r:.3e}")
+
+
+@pytest.mark.parametrize("mode", [True, "all"])
+def test_with_e4m3_matches_fresh_e4m3_model(mode):
+    """DiT.with_e4m3 quantises the resident bf16 weights of a bf16 model; its forward is
+    bit-identical to a model built in e4m3 from the same weights, and the bf16 model it
+    came from is left as it was."""
+    from stream_diffusion_transformer_b200 import model
+    d = dataclasses.replace(zi.FULL, n_noise=1, n_ctx=1, n_main=1)
+    bits = zi.make_weights(d, seed=35, threads=8)
+    fetch = lambda keys: {k: bits[k] for k in keys}
+    base = model.DiT(model.make_config(d), fetch)
+    fresh = model.DiT(model.make_config(d), fetch, fp8=mode)
+    lat = torch.from_numpy(zi.make_latent(d, 1, 16, 16, seed=35)).cuda()
+    txt = torch.from_numpy(zi.make_text(d, 1, 32, seed=35).view(np.int16)).cuda().view(torch.bfloat16)
+    t = torch.tensor([0.4], dtype=torch.float32, device="cuda")
+    y_base = base.forward(lat, t, txt).cpu().numpy()
+    derived = base.with_e4m3(mode)
+    y_derived = derived.forward(lat, t, txt).cpu().numpy()
+    y_fresh = fresh.forward(lat, t, txt).cpu().numpy()
+    np.testing.assert_array_equal(y_derived, y_fresh)
+    np.testing.assert_array_equal(base.forward(lat, t, txt).cpu().numpy(), y_base)
+    assert not np.array_equal(y_derived, y_base)

@@ -21,7 +21,9 @@ and 6,154,908,736 parameters) is checked three ways:
 
 A full-depth forward at a small size (256x256 image: 256 image + 32 text
 tokens, all 34 blocks at full width) is also compared end to end with the
-fp64 oracle.
+fp64 oracle, and so is the 8-step Turbo loop at its own size (1024x1024 image +
+128 text tokens = 4,224 tokens, all 34 blocks): every Euler update along the
+GPU's trajectory, and the transformer output at one mid-loop step end to end.
 """
 import os
 import time
@@ -32,6 +34,7 @@ import pytest
 
 from gpu_util import assert_parity, require_gpu, torch
 import zimage_inputs as zi
+from oracle import scheduler_ref as sch
 from oracle import zimage_ref as ref
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -231,3 +234,48 @@ def test_full_stack_4128_tokens_end_to_end(run):
         worst = min(worst, c)
     print(f"[parity] worst stream cosine over the 34 blocks: {worst:.7f}")
     assert_parity(run["out"], want, rel=1e-1, cos=0.995, what="full stack, 4,128 tokens, end to end")
+
+
+TURBO_TXT = 128
+
+
+def test_turbo_loop_full_size(run):
+    """The 8-step Turbo loop (z-image-turbo-mnn card, "Scheduler": shift 3, t = 1 - sigma',
+    output negated) at its own size, 1024x1024 + 128 text tokens = 4,224 tokens through all
+    34 blocks, checked along the GPU's own trajectory: the CUDA-graph replay the benchmark
+    times ends on the eager loop's latent bit for bit; each of the 8 Euler updates matches
+    the oracle's update of the GPU's latent with the GPU's output; and the transformer output
+    at step 4 (the GPU's own latent after four steps as input) matches the oracle's full
+    forward (fp32) end to end, cosine >= 0.995 (the full-stack bar)."""
+    from stream_diffusion_transformer_b200 import abi, model
+    d, dit = run["d"], run["dit"]
+    n_steps, shift, k = 8, 3.0, 4
+    lat = zi.make_latent(d, 1, LAT, LAT, seed=SEED + 2)
+    txt = zi.make_text(d, 1, TURBO_TXT, seed=SEED + 2)
+    lat_d = torch.from_numpy(lat).cuda()
+    txt_d = torch.from_numpy(txt.view(np.int16)).cuda().view(torch.bfloat16)
+    sig, ts = abi.sigmas(n_steps, shift), abi.timesteps(n_steps, shift)
+    x = lat_d.clone()
+    y = torch.empty_like(x)
+    tt = torch.empty(1, dtype=torch.float32, device="cuda")
+    xs, ys = [lat.copy()], []
+    for i in range(n_steps):
+        tt.fill_(ts[i])
+        dit.forward(x, tt, txt_d, y)
+        ys.append(y.cpu().numpy())
+        model.euler_step(x, y, None, 0.0, sig[i], sig[i + 1])
+        xs.append(x.cpu().numpy())
+    graph = model.DenoiseGraph(dit, lat_d.shape, txt_d, n_steps=n_steps, shift=shift)
+    np.testing.assert_array_equal(graph.run(lat_d).cpu().numpy(), xs[-1])
+    del graph
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    sig_o = sch.sigmas(n_steps, shift)
+    for i in range(n_steps):
+        want = sch.euler_step(xs[i].astype(np.float64), ys[i].astype(np.float64), sig_o[i], sig_o[i + 1])
+        np.testing.assert_allclose(xs[i + 1], want, rtol=1e-5, atol=1e-6 * np.abs(want).max(),
+                                   err_msg=f"Euler update {i}")
+    W = ref.Weights(LazyBits(d, SEED, max(1, min(16, os.cpu_count() or 1))), dtype=np.float32)
+    t_k = np.array([ts[k]], dtype=np.float32)
+    want = ref.model_forward(xs[k], t_k, zi.bf16_bits_to_f32(txt), W, d)
+    assert_parity(ys[k], want, rel=1e-1, cos=0.995, what=f"Turbo loop step {k} (t = {ts[k]:.4f}), 4,224 tokens")
