@@ -13,6 +13,11 @@ TFLOP/s (per block 8SD^2 + 6SDF + 4S^2D, plus embedders and final layer).
 torch.distributed.run); the forward has no exchange step, so there is no
 data-path collective: barriers and the max-over-ranks timing use NCCL.
 
+After the headline timing the same run also times, on the same resident weights,
+the forward with e4m3 projections (e4m3_forwards), the 8-step Turbo loop at
+4,096 + 128 tokens replayed as one CUDA graph, and one CFG step at 2048x2048
+(batch 2 x 16,896 tokens) (workloads); --no-e4m3 / --no-workloads skip them.
+
 --impl reference times the CPU oracle (NumPy, fp64) on the host cores, each
 step one main block of the same 4,128-token workload (a bounded sample).
 
@@ -422,6 +427,68 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if abi.device_status() != 0:
             raise RuntimeError("device pipeline timeout during the e4m3 forwards")
 
+    # ---- the other two workloads of the pages on the same resident weights: the 8-step
+    # Turbo loop (1024x1024 + 128 text tokens, replayed as one CUDA graph) and one CFG step
+    # (2048x2048, batch 2 x (16,384 + 512) tokens, guidance 4); same timing rules, fewer steps
+    workloads = {}
+    if not args.no_workloads:
+        def timed_extra(fn, n):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(local_rank) as clk_w:
+                barrier()
+                torch.cuda.synchronize()
+                g0.record(stream)
+                for _ in range(n):
+                    fn()
+                g1.record(stream)
+                torch.cuda.synchronize()
+                barrier()
+            return max_over_ranks(g0.elapsed_time(g1), world, dev) / n, clk_w.summary()
+
+        n_x = max(1, min(args.steps, 5))
+        txt128 = torch.from_numpy(zi.make_text(d, 1, 128, seed=SEED).view(np.int16)).to(dev).view(torch.bfloat16)
+        graph = model.DenoiseGraph(dit, tuple(lat.shape), txt128, n_steps=8)
+        loop_ms, clk_l = timed_extra(lambda: graph.run(lat), n_x)
+        loop_fl = 8 * forward_flops(d, s_img, 128)
+        workloads["turbo8"] = {"what": f"8-step Turbo loop (shift 3), 1024x1024, {s_img} + 128 tokens, one CUDA graph "
+                                       "(8 forwards and 8 Euler steps)",
+                               "ms_per_loop": loop_ms, "ms_per_forward": loop_ms / 8,
+                               "value": loop_fl * world / (loop_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                               "steps": n_x, "warmup": args.warmup,
+                               "output_finite": bool(torch.isfinite(graph.out).all().item()), "clocks": clk_l}
+        del graph
+        torch.cuda.empty_cache()
+        c_hw, c_txt = 256, 512
+        lat_c1 = torch.from_numpy(zi.make_latent(d, 1, c_hw, c_hw, seed=SEED)).to(dev)
+        lat_c = torch.cat([lat_c1, lat_c1], 0).contiguous()
+        txt_c = torch.cat([torch.from_numpy(zi.make_text(d, 1, c_txt, seed=SEED).view(np.int16)),
+                           torch.from_numpy(zi.make_text(d, 1, c_txt, seed=SEED, uncond=True).view(np.int16))],
+                          0).to(dev).view(torch.bfloat16).contiguous()
+        tt_c = torch.full((2,), T_VALUE, dtype=torch.float32, device=dev)
+        out_c = torch.empty_like(lat_c)
+        x_c = lat_c1.clone()
+        sig = abi.sigmas(8, 3.0)
+
+        def cfg_step():
+            dit.forward(lat_c, tt_c, txt_c, out_c)
+            model.euler_step(x_c, out_c[:1], out_c[1:], 4.0, sig[0], sig[1])
+
+        cfg_ms, clk_c = timed_extra(cfg_step, max(1, min(args.steps, 3)))
+        cfg_fl = forward_flops(d, (c_hw // 2) ** 2, c_txt, batch=2)
+        workloads["cfg"] = {"what": f"CFG step, 2048x2048, batch 2 x ({(c_hw // 2) ** 2} + {c_txt}) tokens, guidance 4 "
+                                    "(one batch-2 forward and the guided Euler step)",
+                            "ms_per_step": cfg_ms, "value": cfg_fl * world / (cfg_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                            "steps": max(1, min(args.steps, 3)), "warmup": args.warmup,
+                            "output_finite": bool(torch.isfinite(x_c).all().item()), "clocks": clk_c}
+        del lat_c, txt_c, out_c, x_c
+        dit._ws.clear()
+        torch.cuda.empty_cache()
+        if abi.device_status() != 0:
+            raise RuntimeError("device pipeline timeout during the Turbo loop or the CFG step")
+
     if rank != 0:
         return
 
@@ -509,6 +576,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clk,
         "output_finite": out_finite,
         "e4m3_forwards": e4m3,
+        "workloads": workloads,
         "published_context": {"ms": 22500.0, "hardware": "Apple M1 Pro", "precision": "int8 ConvRot",
                               "source": "Z-Image-Turbo repackaged for H3ddle, Measured performance"},
     }
@@ -525,8 +593,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     print(json.dumps(line), flush=True)
 
 
-def run_block_workload(args):
-    """One full-width main block over the 4,128-token sequence (profiling-sized case, < 1 GB on the device)."""
+def run_block_workload(args, fp8=False):
+    """One full-width main block over the 4,128-token sequence (profiling-sized case, < 1 GB on the
+    device); fp8 as for DeviceBlock (True: e4m3 QKV and FFN w1|w3, "all": every projection)."""
     import torch
 
     from stream_diffusion_transformer_b200 import abi, model
@@ -536,7 +605,7 @@ def run_block_workload(args):
     gh, gw = LAT_H // 2, LAT_W // 2
     S = gh * gw + S_TXT
     bits = zi.make_weights(d, seed=SEED, keys=model.block_keys("layers.0", True), threads=8)
-    blk = model.DeviceBlock(cfg, "layers.0", bits, True, "cuda")
+    blk = model.DeviceBlock(cfg, "layers.0", bits, True, "cuda", fp8=fp8)
     x = torch.from_numpy(zi.make_stream(d, 1, S, seed=SEED)).cuda()
     c = torch.from_numpy(zi.make_cond(d, 1, seed=SEED)).cuda()
     pos = model.positions(S_TXT, gh, gw)
@@ -554,7 +623,8 @@ def run_block_workload(args):
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     fl = block_flops(S, d.dim, d.ffn)
-    print(json.dumps({"workload": f"one main block, full width, {S} tokens", "ms_per_step": ms,
+    tag = {False: "", True: ", e4m3 QKV and FFN w1|w3", "all": ", every projection in e4m3"}[fp8]
+    print(json.dumps({"workload": f"one main block, full width, {S} tokens{tag}", "ms_per_step": ms,
                       "value": fl / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "steps": args.steps,
                       "kernels": prof.by_kernel(), "device_status": abi.device_status()}), flush=True)
 
@@ -707,17 +777,20 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e4m3", action="store_true", help="skip the e4m3 forwards after the headline timing")
-    ap.add_argument("--workload", choices=["forward", "block", "turbo8", "cfg", "fp8", "fp8all", "oracle"], default="forward",
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the Turbo loop and the CFG step after the headline timing")
+    ap.add_argument("--workload", choices=["forward", "block", "block8", "block8all", "turbo8", "cfg", "fp8", "fp8all",
+                                           "oracle"], default="forward",
                     help="forward: the 4,128-token full forward (the metric); block: one main block of it "
-                         "(a profiling-sized case); turbo8: the 8-step denoising loop at 4,224 tokens; "
+                         "(a profiling-sized case; block8 / block8all: with e4m3 projections); turbo8: the 8-step denoising loop at 4,224 tokens; "
                          "cfg: one guidance step at 2048x2048, batch 2 x 16,896 tokens; fp8 / fp8all: the "
                          "forward with e4m3 projections; oracle: CPU oracle timings on this host")
     args = ap.parse_args()
     if args.workload == "oracle":
         run_oracle_workload(args)
         return
-    if args.workload == "block":
-        run_block_workload(args)
+    if args.workload in ("block", "block8", "block8all"):
+        run_block_workload(args, {"block": False, "block8": True, "block8all": "all"}[args.workload])
         return
     if args.workload == "turbo8":
         run_loop_workload(args)
