@@ -601,6 +601,11 @@ ZI_DEV void gemm_tn_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, 
             tmem_st32(tb + c * 32, v);
           }
           tmem_wait_st();
+          // Each warp group merged its own half of the columns; the SwiGLU epilogue
+          // reads columns of both halves, so all merges finish before any epilogue.
+          tc_fence_before();
+          if (!epi_sync()) break;
+          tc_fence_after();
         }
       }
       if (finish) gemm_epilogue<EPI, BN, F8>(tb, row, row < M, n0, half, ep);
@@ -853,6 +858,11 @@ ZI_DEV void gemm_pair_body(const CUtensorMap& tmA, const CUtensorMap& tmB, int M
             tmem_st32(tb + c * 32, v);
           }
           tmem_wait_st();
+          // Each warp group merged its own half of the columns; the SwiGLU epilogue
+          // reads columns of both halves, so all merges finish before any epilogue.
+          tc_fence_before();
+          if (!epi_sync()) break;
+          tc_fence_after();
         }
       }
       if (finish) gemm_epilogue<EPI, BN, F8>(tb, row, row < M, n0, half, ep);
