@@ -249,7 +249,7 @@ ZI_API int zi_model_forward_trace(const zi_config* cfg, const zi_model_weights* 
  *   y = d_out_uncond ? d_out_uncond + guidance (d_out_cond - d_out_uncond) : d_out_cond
  *   d_x += (sigma_next - sigma) * (-y)          (n fp32 elements)
  * d_out_uncond may be NULL (no CFG; guidance ignored).  n == 0 enqueues nothing and
- * returns ZI_OK whatever the pointers. */
+ * returns ZI_OK whatever the pointers; n above 256 (2^31 - 1) returns ZI_ERR_SHAPE. */
 ZI_API int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond, float guidance, double sigma,
                   double sigma_next, size_t n, zi_stream_t stream);
 
@@ -371,7 +371,8 @@ ZI_API int zi_attention_varlen(const uint16_t* d_qkv, uint16_t* d_out, int batch
  * the result's exponent field.  Maximum relative error 7.5e-5 for x in [-125, 0],
  * below the bf16 rounding the probabilities get next; below -125 (where the result
  * can fall into the denormal range; a masked key's -inf included) it gives a value
- * in [0, 2^-124].  d_x, d_y fp32 [n]; n == 0 enqueues nothing. */
+ * in [0, 2^-124].  d_x, d_y fp32 [n]; n == 0 enqueues nothing; n above 512 (2^31 - 1)
+ * returns ZI_ERR_SHAPE. */
 ZI_API int zi_exp2_poly(const float* d_x, float* d_y, size_t n, zi_stream_t stream);
 
 /* ---------------------------------------------------------------- launch profiling */
