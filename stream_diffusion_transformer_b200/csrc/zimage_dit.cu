@@ -1240,9 +1240,9 @@ int zi_euler_step(float* d_x, const float* d_out_cond, const float* d_out_uncond
                   double sigma_next, size_t n, zi_stream_t stream) {
   if (n == 0) return ZI_OK;  // nothing to do; the pointers of empty arrays may be NULL
   if (!d_x || !d_out_cond) return ZI_ERR_ARG;
+  if ((n + 255) / 256 > size_t(0x7fffffff)) return ZI_ERR_SHAPE;
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
-  if ((n + 255) / 256 > size_t(0x7fffffff)) return ZI_ERR_SHAPE;
   const float dt = float(sigma_next - sigma);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   prof_pre(st);
@@ -1317,11 +1317,11 @@ int zi_watchdog_selftest(int limit_us, zi_stream_t stream) {
 int zi_exp2_poly(const float* d_x, float* d_y, size_t n, zi_stream_t stream) {
   if (n == 0) return ZI_OK;
   if (!d_x || !d_y) return ZI_ERR_ARG;
+  const size_t threads = (n + 1) / 2;
+  if ((threads + 255) / 256 > size_t(0x7fffffff)) return ZI_ERR_SHAPE;
   DevInfo* dev;
   ZI_TRY(current_device(&dev));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t threads = (n + 1) / 2;
-  if ((threads + 255) / 256 > size_t(0x7fffffff)) return ZI_ERR_SHAPE;
   prof_pre(st);
   exp2_poly_kernel<<<unsigned((threads + 255) / 256), 256, 0, st>>>(d_x, d_y, n);
   return launched(ZI_KERNEL_EXP2_TEST, st);

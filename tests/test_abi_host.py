@@ -127,6 +127,13 @@ def test_argument_checks_need_no_gpu(abi):
                           None) == abi.ZI_ERR_SHAPE
     assert L.zi_attention(None, None, 1, 16, 2, None) == abi.ZI_ERR_ARG
     assert L.zi_euler_step(None, None, None, 0.0, 1.0, 0.5, 4, None) == abi.ZI_ERR_ARG
+    huge = 1 << 40  # more than 2^31 - 1 blocks of 256 threads
+    assert L.zi_euler_step(ctypes.c_void_p(16), ctypes.c_void_p(32), None, 0.0, 1.0, 0.5, huge,
+                           None) == abi.ZI_ERR_SHAPE
+    assert L.zi_exp2_poly(ctypes.c_void_p(16), ctypes.c_void_p(32), 2 * huge, None) == abi.ZI_ERR_SHAPE
+    assert L.zi_exp2_poly(None, None, 0, None) == abi.ZI_OK
+    assert L.zi_timesteps(0, 3.0, None) == abi.ZI_ERR_ARG
+    assert L.zi_timesteps(8, 0.0, (ctypes.c_float * 8)()) == abi.ZI_ERR_ARG
     assert L.zi_block_forward(ctypes.byref(c), None, None, None, 1, 16, None, None, None, 0, None) == abi.ZI_ERR_ARG
     assert L.zi_sigmas(0, 3.0, None) == abi.ZI_ERR_ARG
     assert L.zi_watchdog_selftest(0, None) == abi.ZI_ERR_ARG
