@@ -282,17 +282,17 @@ struct TailSched {
 // is read once and the swept one once per group (choose_raster picks the side and
 // the group size from the operands' sizes).
 template <int BM, int BN>
-ZI_DEV void tile_origin(const TailSched& s, int num_m, int tile, int& m0, int& n0) {
+ZI_HD void tile_origin(const TailSched& s, int num_m, int tile, int& m0, int& n0) {
   if (s.group_n) {
     const int per = s.group * num_m;
     const int g = tile / per, r = tile - g * per;
-    const int cols = min(s.group, s.num_n - g * s.group);
+    const int cols = s.group < s.num_n - g * s.group ? s.group : s.num_n - g * s.group;
     n0 = (g * s.group + r % cols) * BN;
     m0 = (r / cols) * BM;
   } else {
     const int per = s.group * s.num_n;
     const int g = tile / per, r = tile - g * per;
-    const int rows = min(s.group, num_m - g * s.group);
+    const int rows = s.group < num_m - g * s.group ? s.group : num_m - g * s.group;
     m0 = (g * s.group + r % rows) * BM;
     n0 = (r / rows) * BN;
   }
@@ -322,6 +322,12 @@ inline void choose_raster(int num_m, int num_n, double a_panel, double b_panel, 
   }
 }
 
+// Units (CTAs, or CTA pairs) a launch needs: one per tile up to G, or one per tail piece.
+inline int sched_units(const TailSched& s, int tiles) {
+  const int u = tiles < s.grid ? tiles : s.grid;
+  return s.tail_items > u ? s.tail_items : u;
+}
+
 inline TailSched make_tail_sched(int tiles, int grid, int kb, bool can_split, int num_n, int group, int group_n) {
   TailSched s{grid, tiles, 1, 0, kb, num_n, group, group_n};
   const int rounds = tiles / grid, rest = tiles - rounds * grid;
@@ -347,8 +353,8 @@ struct WorkWalker {
   const TailSched& s;
   int c, next_dp;
   bool tail_done;
-  ZI_DEV WorkWalker(const TailSched& sched, int cta) : s(sched), c(cta), next_dp(cta), tail_done(false) {}
-  ZI_DEV bool next(WorkItem& w) {
+  ZI_HD WorkWalker(const TailSched& sched, int cta) : s(sched), c(cta), next_dp(cta), tail_done(false) {}
+  ZI_HD bool next(WorkItem& w) {
     if (next_dp < s.dp_tiles) {
       w.tile = next_dp;
       w.kb0 = 0;

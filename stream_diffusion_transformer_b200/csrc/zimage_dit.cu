@@ -190,8 +190,7 @@ int run_gemm(DevInfo* dev, unsigned bit, int kind, const void* A, const void* B,
   choose_raster((M + 127) / 128, N / BN, 128.0 * K * esz, double(BN) * K * esz, group, group_n);
   const TailSched sched =
       make_tail_sched(tiles, dev->sms, K / BK, sk.partials != nullptr, N / BN, group, group_n);
-  int grid = tiles < dev->sms ? tiles : dev->sms;
-  if (sched.tail_items > grid) grid = sched.tail_items;  // fewer tiles than SMs, each cut along K
+  const int grid = sched_units(sched, tiles);
   prof_pre(st);
   kern<<<grid, kGemmThreads, L::kBytes, st>>>(ta, tb, M, ep, sched, sk);
   return launched(kind, st);
@@ -230,8 +229,7 @@ int run_gemm_pair(DevInfo* dev, unsigned bit, int kind, const void* A, const voi
   int group, group_n;
   choose_raster((M + 255) / 256, N / 256, 256.0 * K * esz, 256.0 * K * esz, group, group_n);
   const TailSched sched = make_tail_sched(tiles, pairs, K / BK, sk.partials != nullptr, N / 256, group, group_n);
-  int units = tiles < pairs ? tiles : pairs;
-  if (sched.tail_items > units) units = sched.tail_items;
+  const int units = sched_units(sched, tiles);
   prof_pre(st);
   kern<<<2 * units, kGemmThreads, L::kBytes, st>>>(ta, tb, M, ep, sched, sk);
   return launched(kind, st);
