@@ -14,7 +14,6 @@
 #include <stdint.h>
 
 #define ZI_DEV __device__ __forceinline__
-#define ZI_HD __host__ __device__ __forceinline__  // also callable from host code (schedule checks)
 
 namespace zi {
 

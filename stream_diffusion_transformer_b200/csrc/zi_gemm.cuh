@@ -23,6 +23,9 @@
 #pragma once
 #include "zi_common.cuh"
 
+// Schedule functions callable from host code too (tests/schedule_check.cu runs them on the CPU).
+#define ZI_HD __host__ __device__ __forceinline__
+
 namespace zi {
 
 // Maps a global row of the token buffer to its batch element and to its index
